@@ -1,0 +1,382 @@
+"""Throughput of the merged global-attention layer (HTTM) on B200.
+
+One step = one httm_forward over one VGGT-shaped layer: match, merge, the
+outlier filter, attention and unmerge, with Q/K/V already resident in HBM.
+value = tokens of all ranks / step time (max over ranks); each rank runs its
+own independent layer (weak scaling, no data-path collective).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload vggt_100f]
+    python bench.py --impl reference ...   # the fp64 CPU oracle on a bounded sample
+
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "merged global-attn layer tokens/s at 100/500 frames; % of HBM & tensor roofline"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="vggt_100f")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
+    return ap.parse_args()
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle on a bounded sample
+# ----------------------------------------------------------------------------
+
+def oracle_sample(w, Q, K, V, attn_rows: int, seed: int = 0) -> dict:
+    """The fp64 oracle, as it stands, on one head of the layer: the full plan
+    (matching, merging, outlier filter on that head's share of the budget)
+    plus attention for `attn_rows` seeded query slots, scaled linearly to all
+    slots and all heads.  Returns the extrapolated layer throughput."""
+    import numpy as np
+
+    import oracle.httm_oracle as O
+
+    q, k, v = (t[:1].float().cpu().numpy().astype(np.float64) for t in (Q, K, V))
+    cfg = O.OracleConfig(h=1, T=w.T, P=w.P, d=w.d, n_s=w.n_s, n_t=w.n_t, q_stride=w.q_stride,
+                         kv_stride=w.kv_stride, q_pct=w.q_pct, kv_pct=w.kv_pct, out_pct=w.out_pct,
+                         mode=w.mode, contig_block=w.contig_block)
+    t0 = time.perf_counter()
+    res = O.forward_plan(cfg, q, k, v)
+    t_plan = time.perf_counter() - t0
+    qt = res.restore.q_tilde[0]
+    live = np.concatenate([res.restore.live[0], np.ones(res.restore.n_out[0], dtype=bool)])
+    rows = np.nonzero(live)[0]
+    rng = np.random.default_rng(seed)
+    pick = np.sort(rng.choice(rows, min(attn_rows, rows.shape[0]), replace=False))
+    O.attention(qt[pick[:8]], res.k_means[0], res.v_means[0], cfg.softmax_scale)  # wake the BLAS threads
+    t1 = time.perf_counter()
+    O.attention(qt[pick], res.k_means[0], res.v_means[0], cfg.softmax_scale)
+    t_attn = time.perf_counter() - t1
+    head_s = t_plan + t_attn * rows.shape[0] / pick.shape[0]
+    layer_s = head_s * w.h
+    return {"value": w.N / layer_s, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": (f"head 0 of {w.h}: full plan of all {len(O.block_list(cfg))} blocks "
+                       f"({t_plan:.2f} s) + attention of {pick.shape[0]} of {rows.shape[0]} query slots "
+                       f"({t_attn:.2f} s), scaled linearly to all slots and heads"),
+            "measured_s": t_plan + t_attn}
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region
+# ----------------------------------------------------------------------------
+
+class Clocks:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            sel = ["-i", uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"]
+        except Exception:
+            sel = []
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", *sel, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.flush()
+        self.f.seek(0)
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in self.f.read().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[4:8]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.f.name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------
+# our arm
+# ----------------------------------------------------------------------------
+
+def traffic_record(kernel_file: str):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel source
+    is unchanged since it was captured (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    rec = json.load(open(p)).get(os.path.basename(kernel_file))
+    if not rec:
+        return None
+    sha = hashlib.sha256(open(kernel_file, "rb").read()).hexdigest()[:16]
+    return rec if rec.get("source_sha") == sha else None
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from token_merging_view_b200 import binding as B
+    from token_merging_view_b200.inputs import make_qkv
+    from token_merging_view_b200.workloads import WORKLOADS
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev)
+    w = WORKLOADS[args.workload]
+    Q, K, V = make_qkv(T=w.T, grid=w.grid, h=w.h, d=w.d, seed=w.seed + 1000 * rank, noise_sigma=w.noise_sigma,
+                       max_shift=w.max_shift, dtype=torch.float32 if w.fp32 else torch.bfloat16, device=dev)
+    plan = B.httm_plan(B.LayerConfig.from_workload(w))
+    ws = plan.new_workspace(dev)
+    out = torch.empty_like(Q)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        B.httm_forward(plan, Q, K, V, out=out, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert B.httm_get_device_status(plan, ws) == 0
+    n_out = B.workspace_view(plan, ws, "n_out").cpu()
+    sum_lq = w.h * plan.info.q_slots + int(n_out.sum())
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def timed(fn, steps):
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            fn()
+        b.record(stream)
+        barrier()
+        ms = a.elapsed_time(b)
+        if world > 1:
+            t = torch.tensor([ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms = float(t.item())
+        return ms
+
+    clocks = Clocks(local)
+    plan.profile(True)
+    plan.profile_read()
+    total_ms = timed(step, args.steps)
+    stages = plan.profile_read()
+    plan.profile(False)
+    clk = clocks.stop()
+    launches = plan.launches() * args.steps
+    ms_step = total_ms / args.steps
+    value = world * w.N / (ms_step / 1e3)
+
+    # end to end through the same C ABI call: pinned host Q/K/V in, host out back
+    hQ, hK, hV = (t.cpu().pin_memory() for t in (Q, K, V))
+    hO = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+
+    def e2e_step():
+        Q.copy_(hQ, non_blocking=True)
+        K.copy_(hK, non_blocking=True)
+        V.copy_(hV, non_blocking=True)
+        step()
+        hO.copy_(out, non_blocking=True)
+
+    e2e_step()
+    e2e_steps = max(2, args.steps // 2)
+    e2e_ms = timed(e2e_step, e2e_steps) / e2e_steps
+    h2d = 3 * Q.numel() * Q.element_size()
+    d2h = out.numel() * out.element_size()
+
+    # the dominant kernel: attention on the shortened sequences
+    pk, pk_kind = peaks()
+    att_ms, att_n = stages["attention"]
+    att_avg_ms = att_ms / max(1, att_n)
+    flops = 4.0 * w.d * plan.info.kv_slots * sum_lq
+    achieved = flops / (att_avg_ms / 1e3) / 1e12
+    peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+    import token_merging_view_b200 as pkg
+    att_src = os.path.join(os.path.dirname(pkg.__file__), "csrc", "attn_tc.cu")
+    tr = traffic_record(att_src)
+    roofline = {"bound": "tensor", "kernel": "attention", "achieved": round(achieved, 2), "peak": peak,
+                "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                "peak_kind": f"{pk_kind} bf16 sustained (kernel timed inside a long step)",
+                "traffic": tr["bytes_per_launch"] if tr else None,
+                "algorithmic_flops_per_launch": flops, "avg_launch_ms": round(att_avg_ms, 4)}
+
+    # memory-bound stages against HBM
+    es = 4 if w.fp32 else 2
+    row = w.d * es
+    mem_bytes = {
+        "merge": (3 * w.h * w.N * row + (w.h * plan.info.q_slots + 2 * w.h * plan.info.kv_slots) * row),
+        "unmerge": (w.h * w.N * row + sum_lq * row + w.h * w.N * 4),
+    }
+    hbm = pk["hbm_gbs"]
+    per_step = {k: round(v[0] / args.steps, 4) for k, v in stages.items()}
+    mem_roof = {}
+    for k, b in mem_bytes.items():
+        ms = stages[k][0] / args.steps
+        if ms > 0:
+            mem_roof[k] = {"algorithmic_bytes": b, "ms": round(ms, 4), "GBps": round(b / ms / 1e6, 1),
+                           "frac_of_measured_hbm": round(b / ms / 1e6 / hbm, 4)}
+
+    dense = None
+    if not args.no_dense and rank == 0 and world == 1:
+        dplan = B.httm_plan(B.LayerConfig.from_workload(w, mode=B.HTTM_DENSE))
+        dws = dplan.new_workspace(dev)
+        B.httm_forward(dplan, Q, K, V, out=out, workspace=dws)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        B.httm_forward(dplan, Q, K, V, out=out, workspace=dws, stream=stream)
+        b.record(stream)
+        torch.cuda.synchronize()
+        dms = a.elapsed_time(b)
+        dflops = 4.0 * w.d * w.h * float(w.N) * w.N
+        dense = {"tokens_per_s": round(w.N / (dms / 1e3), 1), "ms": round(dms, 3),
+                 "TFLOPs": round(dflops / (dms / 1e3) / 1e12, 2)}
+        del dws, dplan
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rows = 512 if w.N <= 200_000 else 128
+        cpu = oracle_sample(w, Q, K, V, rows)
+        cpu.pop("measured_s", None)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if not w.fp32 else "f32",
+            "data": "synthetic (seeded blurred-field Q/K/V, VGGT global-attention shapes)",
+            "config": {"workload": w.name, "frames": w.T, "patches_per_frame": w.P, "tokens": w.N, "heads": w.h,
+                       "d_head": w.d, "n_s": w.n_s, "n_t": w.n_t, "q_dst_stride": w.q_stride,
+                       "kv_dst_stride": w.kv_stride, "q_merge_pct": w.q_pct, "kv_merge_pct": w.kv_pct,
+                       "outlier_pct": w.out_pct, "q_rows": sum_lq, "kv_rows_per_head": plan.info.kv_slots,
+                       "parallelism": f"replicas x{world}" if world > 1 else "single",
+                       "l2": f"inputs larger than L2 ({3 * Q.numel() * es / 2**20:.0f} MiB of Q/K/V vs 126 MB)"},
+            "e2e": {"value": round(world * w.N / (e2e_ms / 1e3), 1), "unit": "tokens/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches,
+            "roofline": roofline,
+            "memory_stages": mem_roof,
+            "stage_ms_per_step": per_step,
+            "dense_attention_same_length": dense,
+            "clocks": clk,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def run_reference(args):
+    rank, world, local = dist_env()
+    if rank != 0:
+        return
+    import torch
+
+    from token_merging_view_b200.inputs import make_qkv
+    from token_merging_view_b200.workloads import WORKLOADS
+
+    w = WORKLOADS[args.workload]
+    Q, K, V = make_qkv(T=w.T, grid=w.grid, h=1, d=w.d, seed=w.seed, noise_sigma=w.noise_sigma,
+                       max_shift=w.max_shift, dtype=torch.float32 if w.fp32 else torch.bfloat16)
+    rows = 128
+    for _ in range(args.warmup):
+        oracle_sample(w, Q, K, V, rows)
+    vals, secs, last = [], 0.0, None
+    for i in range(args.steps):
+        last = oracle_sample(w, Q, K, V, rows, seed=i)
+        vals.append(last["value"])
+        secs += last.pop("measured_s")
+    value = statistics.median(vals)
+    cpu = {"value": value, "unit": "tokens/s", "cores": last["cores"], "kind": "oracle", "sample": last["sample"]}
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * secs / args.steps, 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded blurred-field Q/K/V, VGGT global-attention shapes)",
+            "config": {"workload": w.name, "frames": w.T, "tokens": w.N, "heads": w.h, "d_head": w.d},
+            "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "cpu_baseline": cpu}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

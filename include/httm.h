@@ -1,0 +1,243 @@
+/*
+ * httm.h -- C ABI of a B200 (sm_100a) implementation of HTTM's head-wise
+ * temporal token merging around one VGGT-style global-attention layer.
+ *
+ * Method: "HTTM: Head-wise Temporal Token Merging for Faster VGGT"
+ * (papernotes.org note, CVPR 2026).  The layer merges each head's Q/K/V
+ * tokens before the attention kernel and unmerges after it (overall
+ * framework); merging is per head (key design 1), only inside temporal
+ * blocks of n_s patches x n_t frames (key design 2), and a global top-d%
+ * query outlier filter restores badly merged queries (key design 3).
+ *
+ * Conventions shared by every entry point
+ *  - Tensors are row-major [h, N, d_head] with N = T * P and token
+ *    n = t * P + p (p in raster order on the patch grid); element type bf16
+ *    (HTTM_BF16) or fp32 (HTTM_F32).  All tensor pointers are DEVICE
+ *    pointers, 16-byte aligned, owned by the caller.
+ *  - `stream` is a cudaStream_t passed as void*; NULL means the legacy
+ *    default stream.  Entry points that take a stream only enqueue work on
+ *    it: they never synchronise and never copy to the host, unless stated.
+ *  - Host-detectable errors return a status synchronously and enqueue
+ *    nothing.  Errors the device detects (an injected plan that is not a
+ *    valid plan, an index out of bounds, a bounded wait that ran out) set
+ *    bits of a status word kept in the workspace; the kernels skip the bad
+ *    access instead of trapping.  Each forward call clears the word when it
+ *    starts; httm_get_device_status() reads it.
+ *  - Nothing throws across this boundary.  The library allocates no device
+ *    memory except the small block table owned by a plan.
+ */
+#ifndef HTTM_H_
+#define HTTM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  HTTM_OK = 0,
+  HTTM_ERR_ARG = 1,              /* null pointer, bad size or field */
+  HTTM_ERR_UNSUPPORTED = 2,      /* valid request this build does not handle */
+  HTTM_ERR_INFEASIBLE_RATIO = 3, /* r_b exceeds the sources of some block */
+  HTTM_ERR_WORKSPACE = 4,        /* workspace smaller than httm_workspace_bytes() */
+  HTTM_ERR_ALIGN = 5,            /* a pointer is not 16-byte aligned */
+  HTTM_ERR_CUDA = 6,             /* a CUDA runtime call failed */
+  HTTM_ERR_TIMEOUT = 7,          /* device: a bounded wait ran out */
+  HTTM_ERR_DEVICE_BOUNDS = 8,    /* device: an index was out of bounds / plan invalid */
+} httm_status;
+
+typedef enum { HTTM_BF16 = 0, HTTM_F32 = 1 } httm_dtype;
+
+typedef enum {
+  HTTM_HEADWISE_TEMPORAL = 0, /* HTTM: per-head plans inside temporal blocks */
+  HTTM_HEAD_UNIFORM = 1,      /* one plan per block from the head-mean cosine, used by all heads */
+  HTTM_CONTIGUOUS = 2,        /* per-head plans inside runs of contig_block tokens, no reorder */
+  HTTM_DENSE = 3,             /* no merging: plain softmax attention over all N tokens */
+} httm_mode;
+
+/* Device status word bits (httm_get_device_status). */
+#define HTTM_DEV_BAD_PLAN 0x1u    /* an injected plan broke a rule; see httm_forward_with_plan */
+#define HTTM_DEV_BOUNDS 0x2u      /* an index fell outside its buffer */
+#define HTTM_DEV_TIMEOUT 0x4u     /* a bounded device wait ran out */
+
+/*
+ * Layer configuration (plain data).  The knobs are those of the HTTM note's
+ * training-strategy section: n_s spatial tokens x n_t frames per block,
+ * a query merge ratio, a key/value merge ratio and an outlier ratio.
+ *  h, T, P, d_head   heads (<= 64), frames, patch tokens per frame, channels
+ *                    per head; d_head in {16, 64}.  The tensor-core kernels
+ *                    serve bf16 with d_head = 64; other shapes run on
+ *                    CUDA-core kernels (a correctness path for small cases).
+ *  n_s, n_t          block = n_s consecutive patches (raster) x n_t frames;
+ *                    the last region / temporal group may be partial.
+ *  contig_block      block length of HTTM_CONTIGUOUS (ignored otherwise).
+ *  q_dst_stride      the in-block tokens i with i % stride == 0 are the
+ *  kv_dst_stride     destinations, the others sources (>= 2).
+ *  q_merge_pct       r: floor(pct * n_b / 100) sources of each block merge.
+ *  kv_merge_pct
+ *  outlier_pct       d: floor(pct * h * N / 100) queries restored (capped at
+ *                    the number of merged queries).
+ *  softmax_scale     0 selects 1 / sqrt(d_head).
+ */
+typedef struct {
+  int32_t h, T, P, d_head;
+  int32_t dtype; /* httm_dtype */
+  int32_t mode;  /* httm_mode */
+  int32_t n_s, n_t, contig_block;
+  int32_t q_dst_stride, kv_dst_stride;
+  int32_t q_merge_pct, kv_merge_pct, outlier_pct;
+  float softmax_scale;
+} httm_cfg;
+
+typedef struct httm_plan_s* httm_plan_t;
+
+/* Static sizes of a plan (all per head unless stated). */
+typedef struct {
+  int64_t N;              /* tokens */
+  int32_t n_blocks;       /* merge blocks per head */
+  int32_t q_slots;        /* regular query slots R_q = sum_b (n_b - r_b^Q) */
+  int32_t kv_slots;       /* key/value slots L_k = sum_b (n_b - r_b^KV) */
+  int64_t k_out_max;      /* floor(outlier_pct * h * N / 100): outlier budget, all heads */
+  int64_t q_rows_alloc;   /* rows of the shortened-query buffer (all heads, padded) */
+  int64_t ws_q_tilde;     /* workspace byte offsets of the shortened tensors: */
+  int64_t ws_k_tilde;     /*   Q~ rows [q_rows_alloc, d] (regular slots of head hh at */
+  int64_t ws_v_tilde;     /*   hh * q_slots, then per-head outlier runs), K~/V~ [h, L_k, d], */
+  int64_t ws_o_tilde;     /*   O~ laid out like Q~; element type = the input dtype */
+  int64_t ws_n_out;       /* int32 [h]: outliers per head after a forward */
+  int64_t ws_out_base;    /* int32 [h]: first row of each head's outlier run in Q~ */
+  int64_t workspace_bytes;
+} httm_plan_info;
+
+/*
+ * httm_plan: validate `cfg` and build the static block table (key design 2:
+ * temporal reordering into blocks of n_s x n_t) on the host; no device call.
+ * Returns HTTM_ERR_ARG for a bad field, HTTM_ERR_UNSUPPORTED for shapes this
+ * build has no kernel for (d_head not 16/64, a block over 8192 tokens, more
+ * than 64 heads), HTTM_ERR_INFEASIBLE_RATIO when r_b exceeds the sources of
+ * some block.  The first httm_forward* / httm_reorder call uploads the
+ * table to the then-current device (a synchronous copy; make that first call
+ * outside any stream capture) and binds the plan to that device: calls from
+ * another device return HTTM_ERR_ARG.  The plan owns the table until
+ * httm_plan_destroy().
+ */
+httm_status httm_plan(const httm_cfg* cfg, httm_plan_t* out);
+void httm_plan_destroy(httm_plan_t plan);
+httm_status httm_get_plan_info(httm_plan_t plan, httm_plan_info* info);
+
+/* Device workspace bytes httm_forward* needs (caller allocates, >= 256-B aligned). */
+size_t httm_workspace_bytes(httm_plan_t plan);
+
+/*
+ * httm_forward: the merged global-attention layer (overall framework of the
+ * HTTM note): per head and block, bipartite cosine matching of sources to
+ * destinations, top-r mean merging of Q and of K with V following K's plan
+ * (key design 1); the global query outlier filter and restore (key design
+ * 3); softmax(Q~ K~^T * scale) V~ on the shortened sequences; unmerge, which
+ * copies each merged token's output back to its members and undoes the
+ * reorder.  Q, K, V: [h, N, d] inputs; out: [h, N, d] output (same dtype).
+ * HTTM_DENSE computes plain attention of Q, K, V.  Asynchronous on `stream`;
+ * the workspace must not be shared by calls that overlap on the GPU.
+ * Bit-deterministic for identical inputs.
+ */
+httm_status httm_forward(httm_plan_t plan, const void* Q, const void* K, const void* V,
+                         void* out, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Debug exports (all optional DEVICE pointers; NULL skips the export).
+ * Per-token arrays are [h, N] in original token order.
+ */
+typedef struct {
+  int32_t* q_best;    /* original index of the destination each query source chose; -1 on destinations */
+  float* q_score;     /* its cosine (fp32); 0 on destinations */
+  uint8_t* q_merged;  /* 1 if the source merged */
+  int32_t* k_best;    /* the same for the key plan (values follow it) */
+  float* k_score;
+  uint8_t* k_merged;
+  int32_t* q_slot;    /* final query slot: regular slot, or q_slots + rank for an outlier */
+  int32_t* k_slot;    /* key/value slot */
+  float* dev;         /* deviation ||q_n - q~||_2 of eligible queries, 0 otherwise */
+  uint8_t* outlier;   /* the mask M_o */
+  float* q_means;     /* [h, q_slots, d] fp32 query means before the filter */
+  float* q_restored;  /* [h, q_slots, d] fp32 query means after the restore */
+  float* k_means;     /* [h, kv_slots, d] fp32 */
+  float* v_means;     /* [h, kv_slots, d] fp32 */
+} httm_debug;
+
+httm_status httm_forward_debug(httm_plan_t plan, const void* Q, const void* K, const void* V,
+                               void* out, void* workspace, size_t workspace_bytes,
+                               const httm_debug* dbg, void* stream);
+
+/*
+ * A merge plan supplied by the caller (device pointers, [h, N], original
+ * order), which replaces the one the layer would compute, so that merging,
+ * the filter, attention and unmerge can be checked on a given plan.
+ *  q_best/k_best   for each source: original index of its destination (the
+ *                  destination must lie in the same block); ignored on
+ *                  destinations.
+ *  q_merged/k_merged  1 if the source merges; exactly r_b per block.
+ *  outlier         optional M_o (NULL: computed).  Only queries in groups of
+ *                  >= 2 tokens may be set, at most k_out_max in all.
+ * A plan breaking a rule sets HTTM_DEV_BAD_PLAN (the output is then undefined).
+ * In HTTM_HEAD_UNIFORM mode the per-head arrays are used as given.
+ */
+typedef struct {
+  const int32_t* q_best;
+  const uint8_t* q_merged;
+  const int32_t* k_best;
+  const uint8_t* k_merged;
+  const uint8_t* outlier;
+} httm_merge_plan;
+
+httm_status httm_forward_with_plan(httm_plan_t plan, const void* Q, const void* K, const void* V,
+                                   void* out, void* workspace, size_t workspace_bytes,
+                                   const httm_merge_plan* injected, const httm_debug* dbg,
+                                   void* stream);
+
+/*
+ * httm_reorder: temporal reordering (key design 2).  inverse = 0: X in
+ * original order [h, N, d] -> Xb in block order (block after block, each
+ * block frame-major: the n_s-patch region of frame t0, then of t0 + 1, ...).
+ * inverse = 1: the inverse permutation.  X and Xb must not overlap.
+ */
+httm_status httm_reorder(httm_plan_t plan, const void* X, void* Xb, int inverse, void* stream);
+
+/*
+ * Synchronises `stream`, then reads the device status word of `workspace`
+ * into *status (0 = clean; HTTM_DEV_* bits otherwise) and clears it.
+ * Returns HTTM_ERR_DEVICE_BOUNDS / HTTM_ERR_TIMEOUT when bits were set.
+ */
+httm_status httm_get_device_status(httm_plan_t plan, void* workspace, void* stream,
+                                   uint32_t* status);
+
+/* Kernel launches the last httm_forward* call on this plan enqueued. */
+int32_t httm_forward_launches(httm_plan_t plan);
+
+/*
+ * Stage timing.  While enabled, every httm_forward* call on the plan
+ * records a CUDA event pair around each stage on its stream (no host
+ * synchronisation).  httm_profile_read() synchronises on those events, adds
+ * their elapsed times per stage into ms[HTTM_NUM_STAGES] (milliseconds) and
+ * the number of timed launches into launches[HTTM_NUM_STAGES], then forgets
+ * them.  Either output may be NULL.  Host-side only; the plan owns the events.
+ */
+typedef enum {
+  HTTM_STAGE_MATCH = 0,     /* bipartite cosine matching (key design 1) */
+  HTTM_STAGE_MERGE = 1,     /* top-r select, group means, query deviation */
+  HTTM_STAGE_OUTLIER = 2,   /* global top-d% select and restore (key design 3) */
+  HTTM_STAGE_ATTENTION = 3, /* softmax(Q~ K~^T * scale) V~ */
+  HTTM_STAGE_UNMERGE = 4,   /* copy-back in original order */
+  HTTM_STAGE_OTHER = 5,     /* state reset, plan import, debug export */
+  HTTM_NUM_STAGES = 6
+} httm_stage;
+
+httm_status httm_profile_enable(httm_plan_t plan, int enable);
+httm_status httm_profile_read(httm_plan_t plan, float* ms, int32_t* launches);
+
+const char* httm_status_str(httm_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* HTTM_H_ */

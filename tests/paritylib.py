@@ -1,0 +1,164 @@
+"""Helpers for comparing the CUDA path with the fp64 oracle.
+
+Inputs come from the seeded generator and are handed to both sides as the
+same bytes.  Nothing computed by the CUDA path is ever fed to the oracle:
+where fp32 (GPU) and fp64 (oracle) may legitimately pick differently -- a
+destination tied within rounding, a source at the top-r boundary, a query at
+the outlier threshold -- the mismatch is excused only if the ORACLE's own
+values put the two candidates within the stated margin (1e-4).
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle.httm_oracle as O
+from token_merging_view_b200 import binding as B
+from token_merging_view_b200.inputs import make_qkv
+from token_merging_view_b200.workloads import Workload
+
+TIE = 1e-4           # near-tie margin of the plan comparison
+FEAT_REL = 1e-3      # merged features (fp32 exports) vs fp64, per-vector relative L2
+OUT_MAX_ABS = 2e-2   # attention output with the oracle's plan injected
+OUT_REL_L2 = 1e-2
+
+
+def oracle_cfg(w: Workload) -> O.OracleConfig:
+    return O.OracleConfig(h=w.h, T=w.T, P=w.P, d=w.d, n_s=w.n_s, n_t=w.n_t, q_stride=w.q_stride,
+                          kv_stride=w.kv_stride, q_pct=w.q_pct, kv_pct=w.kv_pct, out_pct=w.out_pct,
+                          mode=w.mode, contig_block=w.contig_block)
+
+
+def inputs(w: Workload, device="cuda"):
+    dt = torch.float32 if w.fp32 else torch.bfloat16
+    Q, K, V = make_qkv(T=w.T, grid=w.grid, h=w.h, d=w.d, seed=w.seed, noise_sigma=w.noise_sigma,
+                       max_shift=w.max_shift, dtype=dt, device=device)
+    return Q, K, V
+
+
+def to64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def cpu(x):
+    return {k: v.cpu().numpy() for k, v in x.items()}
+
+
+def oracle_plan_tensors(res: O.OracleResult, device="cuda", mask=True) -> dict:
+    """The oracle's plan in the injection format of httm_forward_with_plan."""
+    def i32(a):
+        return torch.from_numpy(np.ascontiguousarray(a.astype(np.int32))).to(device)
+
+    def u8(a):
+        return torch.from_numpy(np.ascontiguousarray(a.astype(np.uint8))).to(device)
+    d = dict(q_best=i32(res.q_plan.best), q_merged=u8(res.q_plan.merged),
+             k_best=i32(res.k_plan.best), k_merged=u8(res.k_plan.merged))
+    if mask:
+        d["outlier"] = u8(res.mask)
+    return d
+
+
+def compare_best(X64: np.ndarray, plan: O.TensorPlan, g_best: np.ndarray, g_score: np.ndarray) -> int:
+    """Destination choice per source.  Returns the number of excused mismatches;
+    asserts on any other."""
+    src = ~plan.is_dst
+    mism = (g_best != plan.best) & src[None, :]
+    excused = 0
+    for hh, n in zip(*np.nonzero(mism)):
+        t = int(g_best[hh, n])
+        assert 0 <= t < X64.shape[1] and plan.is_dst[t], (hh, n, t)
+        c = O.cosine_similarity(X64[hh, n][None], X64[hh, t][None])[0, 0]
+        gap = plan.score[hh, n] - c
+        assert gap < TIE, f"head {hh} token {n}: GPU dst {t} is {gap:.3g} below the best"
+        excused += 1
+    agree = src[None, :] & ~mism
+    err = np.abs(g_score - plan.score)[agree]
+    assert err.size == 0 or err.max() < 1e-5, f"score error {err.max():.3g}"
+    return excused
+
+
+def compare_merged(blocks, stride: int, pct: int, plan: O.TensorPlan, g_merged: np.ndarray) -> int:
+    """Top-r membership; a mismatch is excused when the oracle's score of that
+    source lies within TIE of its block's r-boundary."""
+    excused = 0
+    h = g_merged.shape[0]
+    for toks in blocks:
+        n_b = toks.shape[0]
+        _, src_i = O.split_dst_src(n_b, stride)
+        r_b = O.merge_count(n_b, pct)
+        st = toks[src_i]
+        for hh in range(h):
+            g = g_merged[hh, st].astype(bool)
+            o = plan.merged[hh, st]
+            assert g.sum() == r_b
+            bad = np.nonzero(g != o)[0]
+            if bad.size == 0:
+                continue
+            sc = np.sort(plan.score[hh, st])[::-1]
+            lo = sc[r_b] if r_b < sc.shape[0] else -np.inf
+            hi = sc[r_b - 1] if r_b > 0 else np.inf
+            for k in bad:
+                s = plan.score[hh, st[k]]
+                assert min(abs(s - lo), abs(s - hi)) < TIE, (hh, st[k], s, lo, hi)
+                excused += 1
+    return excused
+
+
+def rel_rows(g: np.ndarray, o: np.ndarray) -> np.ndarray:
+    num = np.linalg.norm(g - o, axis=-1)
+    den = np.maximum(np.linalg.norm(o, axis=-1), 1e-3)
+    return num / den
+
+
+def compare_mask(res: O.OracleResult, g_mask: np.ndarray) -> int:
+    o = res.mask
+    bad = np.nonzero(g_mask.astype(bool) != o)
+    if bad[0].size == 0:
+        return 0
+    dev = res.dev[res.eligible]
+    k = int(o.sum())
+    thr = np.sort(dev)[::-1][k - 1] if k > 0 else 0.0
+    for hh, n in zip(*bad):
+        assert abs(res.dev[hh, n] - thr) < TIE * max(1.0, thr), (hh, n, res.dev[hh, n], thr)
+    return bad[0].size
+
+
+def bf16_ulps(g: torch.Tensor, o: np.ndarray) -> int:
+    """Max distance in bf16 units between g (bf16) and o rounded to bf16."""
+    ob = torch.from_numpy(o.astype(np.float32)).to(torch.bfloat16)
+    gi = g.cpu().view(torch.int16).to(torch.int32)
+    oi = ob.view(torch.int16).to(torch.int32)
+    return int((gi - oi).abs().max()) if gi.numel() else 0
+
+
+def sample_out_error(res: O.OracleResult, out_g: np.ndarray, cfg: O.OracleConfig, tokens_per_head: int,
+                     seed: int = 0):
+    """Oracle attention for a seeded sample of tokens per head (all tokens if
+    the head is small); returns (max abs error, relative L2 error)."""
+    rng = np.random.default_rng(seed)
+    h, N, _ = out_g.shape
+    errs, nums, dens = [], 0.0, 0.0
+    for hh in range(h):
+        toks = np.arange(N) if N <= tokens_per_head else np.sort(rng.choice(N, tokens_per_head, replace=False))
+        slots = res.restore.slot_final[hh, toks]
+        uniq, inv = np.unique(slots, return_inverse=True)
+        qt = res.restore.q_tilde[hh][uniq]
+        o = O.attention(qt, res.k_means[hh], res.v_means[hh], cfg.softmax_scale)[inv]
+        g = out_g[hh, toks]
+        errs.append(np.abs(g - o).max())
+        nums += float(((g - o) ** 2).sum())
+        dens += float((o ** 2).sum())
+    return max(errs), np.sqrt(nums / dens)
+
+
+def run(plan: B.Plan, Q, K, V, injected=None, debug=True):
+    dbg = B.debug_buffers(plan) if debug else None
+    ws = plan.new_workspace()
+    if injected is not None:
+        out = B.httm_forward_with_plan(plan, Q, K, V, injected, dbg, workspace=ws)
+    elif debug:
+        out = B.httm_forward_debug(plan, Q, K, V, dbg, workspace=ws)
+    else:
+        out = B.httm_forward(plan, Q, K, V, workspace=ws)
+    status = B.httm_get_device_status(plan, ws)
+    return out, (cpu(dbg) if debug else None), ws, status

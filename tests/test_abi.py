@@ -1,0 +1,96 @@
+"""The C ABI library loads on the CPU, exports every symbol include/httm.h
+declares, and its host-side planner validates configurations and sizes the
+layout as the oracle's block table does (no device call is made here)."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle.httm_oracle as O
+from token_merging_view_b200 import binding as B
+from token_merging_view_b200.workloads import WORKLOADS
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "httm.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(httm_[a-z_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = B.load_library()
+    declared = _declared()
+    assert set(declared) == set(B.EXPORTS)
+    for name in declared:
+        assert hasattr(lib, name), name
+        assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
+
+
+def test_status_strings():
+    lib = B.load_library()
+    for s in range(9):
+        assert lib.httm_status_str(s).decode()
+    assert lib.httm_status_str(99).decode() == "unknown status"
+
+
+def _plan_status(**kw):
+    lib = B.load_library()
+    cfg = B.LayerConfig(**{**dict(h=2, T=4, P=64, d_head=16, n_s=16, n_t=4, q_dst_stride=4, kv_dst_stride=4,
+                                   q_merge_pct=50, kv_merge_pct=25, outlier_pct=10), **kw}).to_c()
+    h = ctypes.c_void_p()
+    st = lib.httm_plan(ctypes.byref(cfg), ctypes.byref(h))
+    if st == 0:
+        lib.httm_plan_destroy(h)
+    return st
+
+
+def test_plan_validation():
+    assert _plan_status() == 0
+    assert _plan_status(h=0) == 1                     # HTTM_ERR_ARG
+    assert _plan_status(h=65) == 1
+    assert _plan_status(d_head=32) == 2               # HTTM_ERR_UNSUPPORTED
+    assert _plan_status(mode=7) == 1
+    assert _plan_status(q_dst_stride=1) == 1
+    assert _plan_status(outlier_pct=101) == 1
+    assert _plan_status(q_merge_pct=80) == 3          # r_b = 51 > 48 sources: infeasible
+    assert _plan_status(T=400, n_t=400, n_s=64) == 2  # a block of 25,600 tokens
+    assert _plan_status(softmax_scale=-1.0) == 1
+    lib = B.load_library()
+    assert lib.httm_plan(None, None) == 1
+    assert lib.httm_forward(None, None, None, None, None, None, 0, None) == 1
+
+
+def _oracle_cfg(w):
+    return O.OracleConfig(h=w.h, T=w.T, P=w.P, d=w.d, n_s=w.n_s, n_t=w.n_t, q_stride=w.q_stride,
+                          kv_stride=w.kv_stride, q_pct=w.q_pct, kv_pct=w.kv_pct, out_pct=w.out_pct, mode=w.mode,
+                          contig_block=w.contig_block)
+
+
+@pytest.mark.parametrize("name", sorted(WORKLOADS))
+def test_plan_sizes_match_oracle_block_table(name):
+    w = WORKLOADS[name]
+    plan = B.httm_plan(B.LayerConfig.from_workload(w))
+    ocfg = _oracle_cfg(w)
+    blocks = O.block_list(ocfg)
+    q_slots = sum(b.shape[0] - O.merge_count(b.shape[0], w.q_pct) for b in blocks)
+    kv_slots = sum(b.shape[0] - O.merge_count(b.shape[0], w.kv_pct) for b in blocks)
+    assert plan.info.N == w.N
+    assert plan.info.n_blocks == len(blocks)
+    assert plan.info.q_slots == q_slots
+    assert plan.info.kv_slots == kv_slots
+    assert plan.info.k_out_max == w.out_pct * w.h * w.N // 100
+    assert plan.workspace_bytes > 0
+
+
+def test_contiguous_and_uniform_plans():
+    w = WORKLOADS["vggt_30f"]
+    for mode in (B.HTTM_CONTIGUOUS, B.HTTM_HEAD_UNIFORM):
+        plan = B.httm_plan(B.LayerConfig.from_workload(w, mode=mode))
+        blocks = O.block_list(_oracle_cfg(w.with_(mode=mode)))
+        assert plan.info.n_blocks == len(blocks)
+        assert plan.info.q_slots == sum(b.shape[0] - O.merge_count(b.shape[0], w.q_pct) for b in blocks)

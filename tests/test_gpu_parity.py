@@ -1,0 +1,183 @@
+"""CUDA path vs the fp64 oracle, through the C ABI (needs a B200)."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle.httm_oracle as O
+from tests import paritylib as PL
+from token_merging_view_b200 import binding as B
+from token_merging_view_b200.workloads import CONTIGUOUS, DENSE, HEAD_UNIFORM, WORKLOADS, Workload
+
+pytestmark = pytest.mark.gpu
+
+# 8 frames of the 37 x 37 grid, 4 heads: blocks of 384 / 267 / 256 / 178
+# tokens (partial regions and a partial temporal group), several 128-row tiles
+# with ragged tails.
+MID = Workload("mid_8f", T=8, grid=37, h=4, d=64, fp32=False, n_s=128, n_t=3, q_stride=4, kv_stride=4,
+               q_pct=70, kv_pct=50, out_pct=10, seed=11, noise_sigma=0.3, max_shift=2)
+TINY = WORKLOADS["tiny_4f_8x8"]
+
+
+def _case(w: Workload, **kw):
+    w = w.with_(**kw) if kw else w
+    Q, K, V = PL.inputs(w)
+    plan = B.httm_plan(B.LayerConfig.from_workload(w))
+    cfg = PL.oracle_cfg(w)
+    return w, plan, cfg, (Q, K, V), tuple(PL.to64(t) for t in (Q, K, V))
+
+
+def _full_check(w: Workload, tokens_per_head: int = 1 << 30, max_excused_frac: float = 1e-3):
+    w, plan, cfg, (Q, K, V), (q, k, v) = _case(w)
+    res = O.forward_plan(cfg, q, k, v)
+    # 1. the layer's own plan
+    out, dbg, ws, status = PL.run(plan, Q, K, V)
+    assert status == 0
+    blocks = O.block_list(cfg)
+    ex = PL.compare_best(q, res.q_plan, dbg["q_best"], dbg["q_score"])
+    ex += PL.compare_best(k, res.k_plan, dbg["k_best"], dbg["k_score"])
+    ex += PL.compare_merged(blocks, cfg.q_stride, cfg.q_pct, res.q_plan, dbg["q_merged"])
+    ex += PL.compare_merged(blocks, cfg.kv_stride, cfg.kv_pct, res.k_plan, dbg["k_merged"])
+    assert ex <= max_excused_frac * w.h * w.N
+    # 2. merging, deviation and the filter on the oracle's plan (mask computed)
+    inj = PL.oracle_plan_tensors(res, mask=False)
+    out2, dbg2, ws2, status = PL.run(plan, Q, K, V, injected=inj)
+    assert status == 0
+    assert PL.rel_rows(dbg2["q_means"], res.q_means).max() < PL.FEAT_REL
+    assert PL.rel_rows(dbg2["k_means"], res.k_means).max() < PL.FEAT_REL
+    assert PL.rel_rows(dbg2["v_means"], res.v_means).max() < PL.FEAT_REL
+    kt = B.workspace_view(plan, ws2, "k")[: w.h * plan.info.kv_slots]
+    vt = B.workspace_view(plan, ws2, "v")[: w.h * plan.info.kv_slots]
+    if not w.fp32:
+        assert PL.bf16_ulps(kt, res.k_means.reshape(-1, w.d)) <= 1
+        assert PL.bf16_ulps(vt, res.v_means.reshape(-1, w.d)) <= 1
+    assert np.all(np.abs(dbg2["dev"] - res.dev) <= 1e-4 * np.maximum(1.0, res.dev))
+    n_mask_ex = PL.compare_mask(res, dbg2["outlier"])
+    assert n_mask_ex <= max(2, max_excused_frac * w.h * w.N)
+    # 3. the whole layer on the oracle's plan and mask
+    inj["outlier"] = PL.oracle_plan_tensors(res)["outlier"]
+    out3, dbg3, ws3, status = PL.run(plan, Q, K, V, injected=inj)
+    assert status == 0
+    live = res.restore.live
+    assert PL.rel_rows(dbg3["q_restored"][live], res.restore.means[live]).max() < PL.FEAT_REL
+    assert np.array_equal(B.workspace_view(plan, ws3, "n_out").cpu().numpy(), res.restore.n_out)
+    assert np.array_equal(dbg3["q_slot"], res.restore.slot_final)
+    assert np.array_equal(dbg3["outlier"].astype(bool), res.mask)
+    mx, rl2 = PL.sample_out_error(res, PL.to64(out3), cfg, tokens_per_head)
+    assert mx <= PL.OUT_MAX_ABS and rl2 <= PL.OUT_REL_L2, (mx, rl2)
+    # the layer's own end-to-end output stays within the same bound
+    mx, rl2 = PL.sample_out_error(res, PL.to64(out), cfg, min(tokens_per_head, 256), seed=1)
+    return ex, n_mask_ex, (mx, rl2)
+
+
+def test_tiny_fp32_layer_exact_plan():
+    ex, mex, _ = _full_check(TINY, max_excused_frac=0.0)
+    assert ex == 0 and mex == 0
+
+
+def test_mid_layer():
+    _full_check(MID)
+
+
+def test_mid_layer_contiguous_blocks():
+    _full_check(MID.with_(mode=CONTIGUOUS, contig_block=384))
+
+
+def test_mid_layer_head_uniform():
+    _full_check(MID.with_(mode=HEAD_UNIFORM))
+
+
+@pytest.mark.parametrize("kw", [dict(out_pct=0), dict(out_pct=100), dict(q_pct=0, kv_pct=0),
+                                dict(T=1, n_t=1), dict(q_stride=8, q_pct=85), dict(n_s=100, n_t=2)])
+def test_mid_layer_edge_cases(kw):
+    _full_check(MID.with_(**kw))
+
+
+def test_vggt_30f_layer():
+    _full_check(WORKLOADS["vggt_30f"], tokens_per_head=512)
+
+
+@pytest.mark.slow
+def test_vggt_100f_layer_sampled():
+    _full_check(WORKLOADS["vggt_100f"], tokens_per_head=128)
+
+
+def test_reorder_matches_oracle():
+    for w in (TINY, MID, MID.with_(mode=CONTIGUOUS, contig_block=500)):
+        _, plan, cfg, (Q, _, _), (q, _, _) = _case(w)
+        Xb = B.httm_reorder(plan, Q)
+        want = O.reorder(q, O.block_list(cfg))
+        assert np.array_equal(PL.to64(Xb), want)
+        back = B.httm_reorder(plan, Xb, inverse=True)
+        assert torch.equal(back, Q)
+
+
+def test_dense_mode_and_unmerged_layer():
+    w = MID.with_(T=2, h=2)
+    _, plan, cfg, (Q, K, V), (q, k, v) = _case(w, mode=DENSE)
+    out = B.httm_forward(plan, Q, K, V)
+    want = O.forward(PL.oracle_cfg(w.with_(mode=DENSE)), q, k, v).out
+    g = PL.to64(out)
+    assert np.abs(g - want).max() <= PL.OUT_MAX_ABS
+    assert np.linalg.norm(g - want) / np.linalg.norm(want) <= PL.OUT_REL_L2
+    # r = 0: the merged layer reduces to dense attention
+    _, plan0, _, _, _ = _case(w, q_pct=0, kv_pct=0)
+    out0 = B.httm_forward(plan0, Q, K, V)
+    g0 = PL.to64(out0)
+    assert np.abs(g0 - want).max() <= PL.OUT_MAX_ABS
+
+
+def test_identical_and_zero_tokens():
+    w = MID.with_(T=3, h=2)
+    _, plan, cfg, (Q, K, V), _ = _case(w)
+    Q = torch.zeros_like(Q)
+    K = K[:, :1].expand_as(K).contiguous()          # every key identical
+    q, k, v = (PL.to64(t) for t in (Q, K, V))
+    res = O.forward_plan(cfg, q, k, v)
+    out, dbg, ws, status = PL.run(plan, Q, K, V)
+    assert status == 0
+    assert np.array_equal(dbg["q_best"], res.q_plan.best) and np.array_equal(dbg["k_best"], res.k_plan.best)
+    assert np.array_equal(dbg["q_merged"].astype(bool), res.q_plan.merged)
+    assert np.array_equal(dbg["k_merged"].astype(bool), res.k_plan.merged)
+    assert np.all(dbg["dev"] == 0.0)
+
+
+def test_deterministic():
+    _, plan, _, (Q, K, V), _ = _case(MID)
+    a, da, _, _ = PL.run(plan, Q, K, V)
+    b, db, _, _ = PL.run(plan, Q, K, V)
+    assert torch.equal(a, b)
+    for key in da:
+        assert np.array_equal(da[key], db[key], equal_nan=True), key
+
+
+def test_invalid_injected_plan_sets_status():
+    w, plan, cfg, (Q, K, V), (q, k, v) = _case(MID.with_(T=3, h=2))
+    res = O.forward_plan(cfg, q, k, v)
+    inj = PL.oracle_plan_tensors(res, mask=False)
+    inj["q_merged"] = torch.zeros_like(inj["q_merged"])        # wrong merge count in every block
+    _, _, _, status = PL.run(plan, Q, K, V, injected=inj, debug=False)
+    assert status & B.HTTM_DEV_BAD_PLAN
+    inj = PL.oracle_plan_tensors(res, mask=False)
+    inj["k_best"] = torch.where(inj["k_best"] >= 0, (inj["k_best"] + 1) % w.N, inj["k_best"])  # a non-dst target
+    _, _, _, status = PL.run(plan, Q, K, V, injected=inj, debug=False)
+    assert status & B.HTTM_DEV_BAD_PLAN
+    # a clean call afterwards reports a clean status
+    _, _, _, status = PL.run(plan, Q, K, V, debug=False)
+    assert status == 0
+
+
+def test_host_errors():
+    _, plan, _, (Q, K, V), _ = _case(MID.with_(T=2, h=2))
+    ws = plan.new_workspace()
+    with pytest.raises(B.HttmError) as e:
+        B.httm_forward(plan, Q, K, V, workspace=ws[: plan.workspace_bytes // 2])
+    assert e.value.status == 4                                   # HTTM_ERR_WORKSPACE
+    with pytest.raises(B.HttmError) as e:
+        B.httm_forward(plan, Q, K, V, workspace=ws[1:])
+    assert e.value.status == 5                                   # HTTM_ERR_ALIGN
+    Qm = torch.empty(Q.numel() + 8, dtype=Q.dtype, device=Q.device)[1:1 + Q.numel()].view(Q.shape)
+    with pytest.raises(B.HttmError) as e:
+        B.httm_forward(plan, Qm, K, V, workspace=ws)
+    assert e.value.status == 5

@@ -1,0 +1,519 @@
+// Host side of the C ABI: validation, the static block table (key design 2
+// of the HTTM note: blocks of n_s patches x n_t frames), the workspace layout
+// and the launch sequence of one merged global-attention layer.
+#include <algorithm>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "../../include/httm.h"
+#include "internal.h"
+#include "launch.h"
+
+using namespace httm;
+
+struct httm_plan_s {
+  httm_cfg cfg;
+  Dims dims;
+  bool fp32;
+  int device = -1;
+  std::vector<BlockDesc> blocks_h;
+  BlockDesc* blocks_d = nullptr;
+  int4* match_items_d = nullptr;
+  int n_match_items = 0;
+  Workspace ws;
+  int launches = 0;
+  std::vector<int4> items_h;
+  // stage timing
+  bool profile = false;
+  struct Rec { int stage; int n; cudaEvent_t a, b; };
+  std::vector<Rec> recs;
+  std::vector<cudaEvent_t> pool;
+};
+
+namespace {
+cudaEvent_t pool_event(httm_plan_s* p) {
+  if (!p->pool.empty()) {
+    cudaEvent_t e = p->pool.back();
+    p->pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+
+// Brackets the launches of one stage with an event pair when profiling.
+struct StageTimer {
+  httm_plan_s* p;
+  cudaStream_t s;
+  int stage, n;
+  cudaEvent_t a = nullptr;
+  StageTimer(httm_plan_s* p_, cudaStream_t s_, int stage_, int n_) : p(p_), s(s_), stage(stage_), n(n_) {
+    if (p->profile && (a = pool_event(p)) != nullptr) cudaEventRecord(a, s);
+  }
+  ~StageTimer() {
+    if (!a) return;
+    cudaEvent_t b = pool_event(p);
+    if (!b) {
+      p->pool.push_back(a);
+      return;
+    }
+    cudaEventRecord(b, s);
+    p->recs.push_back({stage, n, a, b});
+  }
+};
+}  // namespace
+
+namespace httm {
+cudaError_t launch_attention_simt(const Dims& dims, bool fp32, const void* q, const void* k, const void* v,
+                                  void* o, int Lk, const Buffers& buf, cudaStream_t s);
+bool attention_tc_supported(const Dims& dims, bool fp32);
+cudaError_t launch_attention_tc(const Dims& dims, const void* q, const void* k, const void* v, void* o,
+                                int Lk, const Buffers& buf, cudaStream_t s);
+bool match_tc_supported(const Dims& dims, bool fp32);
+}  // namespace httm
+
+namespace {
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+Workspace layout(const Dims& d, bool fp32) {
+  Workspace w{};
+  const size_t es = fp32 ? 4 : 2;
+  const size_t hN = (size_t)d.h * d.N;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  w.state = take(sizeof(DevState));
+  w.hist = take(3ull * kHistBins * 4);
+  w.chunk = take((size_t)d.h * d.nchunk_per_head * 16);
+  w.n_out = take((size_t)d.h * 4);
+  w.out_base = take((size_t)d.h * 4);
+  w.items = take((size_t)d.max_items * 16);
+  w.q_best = take((size_t)d.h * d.q_src * 4);
+  w.q_score = take((size_t)d.h * d.q_src * 4);
+  w.q_merged = take((size_t)d.h * d.q_src);
+  w.k_best = take((size_t)d.h * d.k_src * 4);
+  w.k_score = take((size_t)d.h * d.k_src * 4);
+  w.k_merged = take((size_t)d.h * d.k_src);
+  w.q_slot = take(hN * 4);
+  w.keys = take(hN * 4);
+  w.mask = take(hN);
+  w.q_members = take(hN * 4);
+  w.q_gstart = take((size_t)d.h * d.q_slots * 4);
+  w.q_gcount = take((size_t)d.h * d.q_slots * 4);
+  w.q_tilde = take((size_t)d.q_rows_alloc * d.d * es);
+  w.k_tilde = take((size_t)d.h * d.k_slots * d.d * es);
+  w.v_tilde = take((size_t)d.h * d.k_slots * d.d * es);
+  w.o_tilde = take((size_t)d.q_rows_alloc * d.d * es);
+  w.total = off;
+  return w;
+}
+
+Buffers resolve(const Workspace& w, void* base) {
+  char* p = static_cast<char*>(base);
+  Buffers b{};
+  b.state = reinterpret_cast<DevState*>(p + w.state);
+  b.hist = reinterpret_cast<uint32_t*>(p + w.hist);
+  b.chunk = reinterpret_cast<uint32_t*>(p + w.chunk);
+  b.n_out = reinterpret_cast<int32_t*>(p + w.n_out);
+  b.out_base = reinterpret_cast<int32_t*>(p + w.out_base);
+  b.items = reinterpret_cast<int4*>(p + w.items);
+  b.q_best = reinterpret_cast<int32_t*>(p + w.q_best);
+  b.q_score = reinterpret_cast<float*>(p + w.q_score);
+  b.q_merged = reinterpret_cast<uint8_t*>(p + w.q_merged);
+  b.k_best = reinterpret_cast<int32_t*>(p + w.k_best);
+  b.k_score = reinterpret_cast<float*>(p + w.k_score);
+  b.k_merged = reinterpret_cast<uint8_t*>(p + w.k_merged);
+  b.q_slot = reinterpret_cast<int32_t*>(p + w.q_slot);
+  b.keys = reinterpret_cast<uint32_t*>(p + w.keys);
+  b.mask = reinterpret_cast<uint8_t*>(p + w.mask);
+  b.q_members = reinterpret_cast<int32_t*>(p + w.q_members);
+  b.q_gstart = reinterpret_cast<int32_t*>(p + w.q_gstart);
+  b.q_gcount = reinterpret_cast<int32_t*>(p + w.q_gcount);
+  b.q_tilde = p + w.q_tilde;
+  b.k_tilde = p + w.k_tilde;
+  b.v_tilde = p + w.v_tilde;
+  b.o_tilde = p + w.o_tilde;
+  return b;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// The first call that needs the device uploads the block table and the
+// matching work list to the current device (synchronously) and binds the
+// plan to that device; later calls must come from the same device.
+httm_status check_device(httm_plan_s* plan) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return HTTM_ERR_CUDA;
+  if (plan->device < 0) {
+    if (plan->dims.mode != HTTM_DENSE) {
+      const size_t nb = plan->blocks_h.size() * sizeof(BlockDesc);
+      const size_t ni = std::max<size_t>(1, plan->items_h.size()) * sizeof(int4);
+      if (cudaMalloc(&plan->blocks_d, nb) != cudaSuccess ||
+          cudaMemcpy(plan->blocks_d, plan->blocks_h.data(), nb, cudaMemcpyHostToDevice) != cudaSuccess ||
+          cudaMalloc(&plan->match_items_d, ni) != cudaSuccess ||
+          (!plan->items_h.empty() &&
+           cudaMemcpy(plan->match_items_d, plan->items_h.data(), plan->items_h.size() * sizeof(int4),
+                      cudaMemcpyHostToDevice) != cudaSuccess)) {
+        if (plan->blocks_d) cudaFree(plan->blocks_d);
+        if (plan->match_items_d) cudaFree(plan->match_items_d);
+        plan->blocks_d = nullptr;
+        plan->match_items_d = nullptr;
+        return HTTM_ERR_CUDA;
+      }
+    }
+    plan->device = dev;
+  }
+  return dev == plan->device ? HTTM_OK : HTTM_ERR_ARG;
+}
+
+#define HTTM_LAUNCH(expr)                             \
+  do {                                                \
+    cudaError_t e_ = (expr);                          \
+    ++launches;                                       \
+    if (e_ != cudaSuccess) return HTTM_ERR_CUDA;      \
+  } while (0)
+
+httm_status attention(const httm_plan_s* plan, const void* q, const void* k, const void* v, void* o, int Lk,
+                      const Buffers& buf, cudaStream_t s) {
+  cudaError_t e;
+  if (attention_tc_supported(plan->dims, plan->fp32)) e = launch_attention_tc(plan->dims, q, k, v, o, Lk, buf, s);
+  else e = launch_attention_simt(plan->dims, plan->fp32, q, k, v, o, Lk, buf, s);
+  return e == cudaSuccess ? HTTM_OK : HTTM_ERR_CUDA;
+}
+
+httm_status forward_impl(httm_plan_s* plan, const void* Q, const void* K, const void* V, void* out, void* ws,
+                         size_t ws_bytes, const httm_merge_plan* inj, const httm_debug* dbg, void* stream) {
+  if (!plan || !Q || !K || !V || !out || !ws) return HTTM_ERR_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(out)) return HTTM_ERR_ALIGN;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return HTTM_ERR_ALIGN;
+  if (ws_bytes < plan->ws.total) return HTTM_ERR_WORKSPACE;
+  if (inj) {
+    const bool any = inj->q_best || inj->q_merged || inj->k_best || inj->k_merged;
+    const bool all = inj->q_best && inj->q_merged && inj->k_best && inj->k_merged;
+    if (any && !all) return HTTM_ERR_ARG;
+    if (plan->dims.mode == HTTM_DENSE) return HTTM_ERR_ARG;
+  }
+  httm_status st = check_device(plan);
+  if (st != HTTM_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const Dims& dims = plan->dims;
+  const bool fp32 = plan->fp32;
+  Buffers buf = resolve(plan->ws, ws);
+  Debug dd{};
+  if (dbg) {
+    dd = Debug{dbg->q_best, dbg->q_score, dbg->q_merged, dbg->k_best, dbg->k_score, dbg->k_merged,
+               dbg->q_slot, dbg->k_slot, dbg->dev, dbg->outlier, dbg->q_means, dbg->q_restored,
+               dbg->k_means, dbg->v_means};
+  }
+  int launches = 0;
+  {
+    StageTimer t(plan, s, HTTM_STAGE_OTHER, dims.mode == HTTM_DENSE ? 2 : 1);
+    HTTM_LAUNCH(launch_zero_state(dims, buf, s));
+    if (dims.mode == HTTM_DENSE) HTTM_LAUNCH(launch_dense_items(dims, buf, s));
+  }
+  if (dims.mode == HTTM_DENSE) {
+    StageTimer t(plan, s, HTTM_STAGE_ATTENTION, 1);
+    st = attention(plan, Q, K, V, out, dims.N, buf, s);
+    ++launches;
+    plan->launches = launches;
+    return st;
+  }
+  const bool plan_inj = inj && inj->q_best;
+  const bool mask_inj = inj && inj->outlier;
+  if (plan_inj || mask_inj) {
+    StageTimer t(plan, s, HTTM_STAGE_OTHER, 1);
+    Inject ii{inj->q_best, inj->q_merged, inj->k_best, inj->k_merged, inj->outlier};
+    HTTM_LAUNCH(launch_import_plan(dims, plan->blocks_d, ii, buf, s));
+  }
+  if (!plan_inj) {
+    StageTimer t(plan, s, HTTM_STAGE_MATCH, 1);
+    cudaError_t e = cudaErrorNotSupported;
+    if (match_tc_supported(dims, fp32))
+      e = launch_match_tc(dims, plan->blocks_d, plan->match_items_d, plan->n_match_items, Q, K, buf, s);
+    else
+      e = launch_match_simt(dims, fp32, plan->blocks_d, plan->match_items_d, plan->n_match_items, Q, K, buf, s);
+    ++launches;
+    if (e != cudaSuccess) return HTTM_ERR_CUDA;
+  }
+  {
+    StageTimer t(plan, s, HTTM_STAGE_MERGE, 2);
+    HTTM_LAUNCH(launch_merge(dims, fp32, plan->blocks_d, true, plan_inj, Q, nullptr, buf, dd, s));
+    HTTM_LAUNCH(launch_merge(dims, fp32, plan->blocks_d, false, plan_inj, K, V, buf, dd, s));
+  }
+  {
+    StageTimer t(plan, s, HTTM_STAGE_OUTLIER, mask_inj ? 4 : 6);
+    HTTM_LAUNCH(launch_outlier(dims, fp32, Q, mask_inj, buf, s));
+    launches += mask_inj ? 2 : 4;  // count, scan, emit, plus two histogram passes
+    HTTM_LAUNCH(launch_restore(dims, fp32, plan->blocks_d, Q, buf, dd, s));
+  }
+  {
+    StageTimer t(plan, s, HTTM_STAGE_ATTENTION, 1);
+    st = attention(plan, buf.q_tilde, buf.k_tilde, buf.v_tilde, buf.o_tilde, dims.k_slots, buf, s);
+    ++launches;
+    if (st != HTTM_OK) return st;
+  }
+  {
+    StageTimer t(plan, s, HTTM_STAGE_UNMERGE, 1);
+    HTTM_LAUNCH(launch_unmerge(dims, fp32, buf, out, s));
+  }
+  if (dbg) {
+    StageTimer t(plan, s, HTTM_STAGE_OTHER, 1);
+    HTTM_LAUNCH(launch_export(dims, plan->blocks_d, buf, dd, s));
+  }
+  plan->launches = launches;
+  return HTTM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* httm_status_str(httm_status s) {
+  switch (s) {
+    case HTTM_OK: return "ok";
+    case HTTM_ERR_ARG: return "invalid argument";
+    case HTTM_ERR_UNSUPPORTED: return "unsupported configuration";
+    case HTTM_ERR_INFEASIBLE_RATIO: return "merge ratio exceeds the sources of a block";
+    case HTTM_ERR_WORKSPACE: return "workspace too small";
+    case HTTM_ERR_ALIGN: return "pointer not aligned";
+    case HTTM_ERR_CUDA: return "CUDA runtime error";
+    case HTTM_ERR_TIMEOUT: return "device wait timed out";
+    case HTTM_ERR_DEVICE_BOUNDS: return "device bounds / plan check failed";
+  }
+  return "unknown status";
+}
+
+httm_status httm_plan(const httm_cfg* cfg, httm_plan_t* out) {
+  if (!cfg || !out) return HTTM_ERR_ARG;
+  *out = nullptr;
+  const httm_cfg c = *cfg;
+  if (c.h < 1 || c.h > 64 || c.T < 1 || c.P < 1) return HTTM_ERR_ARG;
+  if (c.dtype != HTTM_BF16 && c.dtype != HTTM_F32) return HTTM_ERR_ARG;
+  if (c.mode < HTTM_HEADWISE_TEMPORAL || c.mode > HTTM_DENSE) return HTTM_ERR_ARG;
+  if (c.d_head != 16 && c.d_head != 64) return HTTM_ERR_UNSUPPORTED;
+  if (c.softmax_scale < 0.f) return HTTM_ERR_ARG;
+  const long long N = (long long)c.T * c.P;
+  if (N > (1ll << 30) || (long long)c.h * N > (1ll << 31) - 1) return HTTM_ERR_UNSUPPORTED;
+  if (c.mode != HTTM_DENSE) {
+    if (c.q_dst_stride < 2 || c.kv_dst_stride < 2) return HTTM_ERR_ARG;
+    if (c.q_merge_pct < 0 || c.q_merge_pct > 100 || c.kv_merge_pct < 0 || c.kv_merge_pct > 100) return HTTM_ERR_ARG;
+    if (c.outlier_pct < 0 || c.outlier_pct > 100) return HTTM_ERR_ARG;
+    if (c.mode == HTTM_CONTIGUOUS ? c.contig_block < 1 : (c.n_s < 1 || c.n_t < 1)) return HTTM_ERR_ARG;
+  }
+  httm_plan_s* p = new (std::nothrow) httm_plan_s();
+  if (!p) return HTTM_ERR_ARG;
+  p->cfg = c;
+  p->fp32 = c.dtype == HTTM_F32;
+  Dims& d = p->dims;
+  d = Dims{};
+  d.h = c.h;
+  d.N = (int32_t)N;
+  d.P = c.P;
+  d.d = c.d_head;
+  d.mode = c.mode;
+  d.n_s = c.n_s;
+  d.n_t = c.n_t;
+  d.contig = c.contig_block;
+  d.q_stride = c.q_dst_stride;
+  d.kv_stride = c.kv_dst_stride;
+  d.scale = c.softmax_scale > 0.f ? c.softmax_scale : 1.0f / sqrtf((float)c.d_head);
+  d.nchunk_per_head = (int32_t)((N + kChunk - 1) / kChunk);
+  if (c.mode == HTTM_DENSE) {
+    d.max_items = (int32_t)(c.h * ((N + kAttnRows - 1) / kAttnRows));
+  } else {
+    std::vector<BlockDesc>& B = p->blocks_h;
+    auto add = [&](int base, int s, int n_b) {
+      BlockDesc b{};
+      b.base = base;
+      b.s = s;
+      b.n_b = n_b;
+      B.push_back(b);
+    };
+    if (c.mode == HTTM_CONTIGUOUS) {
+      for (long long s0 = 0; s0 < N; s0 += c.contig_block) {
+        const int nb = (int)std::min<long long>(c.contig_block, N - s0);
+        add((int)s0, nb, nb);
+      }
+      d.R = 0;
+    } else {
+      const int G = (c.T + c.n_t - 1) / c.n_t;
+      const int R = (c.P + c.n_s - 1) / c.n_s;
+      d.R = R;
+      for (int g = 0; g < G; ++g) {
+        const int t0 = g * c.n_t, tg = std::min(c.n_t, c.T - t0);
+        for (int j = 0; j < R; ++j) {
+          const int p0 = j * c.n_s, sj = std::min(c.n_s, c.P - p0);
+          add(t0 * c.P + p0, sj, tg * sj);
+        }
+      }
+    }
+    int tok = 0, qs = 0, ks = 0, qsl = 0, ksl = 0;
+    for (BlockDesc& b : B) {
+      if (b.n_b > 8192) {
+        delete p;
+        return HTTM_ERR_UNSUPPORTED;
+      }
+      b.tok_off = tok;
+      b.q_ndst = (b.n_b + c.q_dst_stride - 1) / c.q_dst_stride;
+      b.k_ndst = (b.n_b + c.kv_dst_stride - 1) / c.kv_dst_stride;
+      b.q_r = (int)(((long long)c.q_merge_pct * b.n_b) / 100);
+      b.k_r = (int)(((long long)c.kv_merge_pct * b.n_b) / 100);
+      if (b.q_r > b.n_b - b.q_ndst || b.k_r > b.n_b - b.k_ndst) {
+        delete p;
+        return HTTM_ERR_INFEASIBLE_RATIO;
+      }
+      b.q_src_off = qs;
+      b.k_src_off = ks;
+      b.q_slot_off = qsl;
+      b.k_slot_off = ksl;
+      tok += b.n_b;
+      qs += b.n_b - b.q_ndst;
+      ks += b.n_b - b.k_ndst;
+      qsl += b.n_b - b.q_r;
+      ksl += b.n_b - b.k_r;
+      d.max_ndst = std::max(d.max_ndst, std::max(b.q_ndst, b.k_ndst));
+      d.max_nsrc = std::max(d.max_nsrc, std::max(b.n_b - b.q_ndst, b.n_b - b.k_ndst));
+      d.max_nb = std::max(d.max_nb, b.n_b);
+    }
+    d.nblk = (int32_t)B.size();
+    d.q_src = qs;
+    d.k_src = ks;
+    d.q_slots = qsl;
+    d.k_slots = ksl;
+    d.k_out_max = ((long long)c.outlier_pct * c.h * N) / 100;
+    d.out_base = (long long)align_up((size_t)c.h * qsl, kAttnRows);
+    d.q_rows_alloc = d.out_base + d.k_out_max + (long long)kAttnRows * (c.h + 1);
+    d.max_items = (int32_t)(c.h * ((qsl + kAttnRows - 1) / kAttnRows) + (d.k_out_max + kAttnRows - 1) / kAttnRows + c.h);
+    // matching work: 128-source tiles of every (tensor, block), costliest first
+    std::vector<int4> items;
+    for (int t = 0; t < 2; ++t)
+      for (int bi = 0; bi < d.nblk; ++bi) {
+        const BlockDesc& b = B[bi];
+        const int ns = b.n_b - (t == 0 ? b.q_ndst : b.k_ndst);
+        for (int s0 = 0; s0 < ns; s0 += 128) items.push_back(make_int4(t, bi, s0, std::min(128, ns - s0)));
+      }
+    std::stable_sort(items.begin(), items.end(), [&](const int4& a, const int4& b) {
+      const int ca = a.x == 0 ? B[a.y].q_ndst : B[a.y].k_ndst;
+      const int cb = b.x == 0 ? B[b.y].q_ndst : B[b.y].k_ndst;
+      return ca > cb;
+    });
+    p->n_match_items = (int)items.size();
+    p->items_h = std::move(items);
+  }
+  p->ws = layout(d, p->fp32);
+  *out = p;
+  return HTTM_OK;
+}
+
+void httm_plan_destroy(httm_plan_t plan) {
+  if (!plan) return;
+  for (auto& r : plan->recs) {
+    cudaEventDestroy(r.a);
+    cudaEventDestroy(r.b);
+  }
+  for (cudaEvent_t e : plan->pool) cudaEventDestroy(e);
+  if (plan->blocks_d) cudaFree(plan->blocks_d);
+  if (plan->match_items_d) cudaFree(plan->match_items_d);
+  delete plan;
+}
+
+size_t httm_workspace_bytes(httm_plan_t plan) { return plan ? plan->ws.total : 0; }
+
+httm_status httm_get_plan_info(httm_plan_t plan, httm_plan_info* info) {
+  if (!plan || !info) return HTTM_ERR_ARG;
+  const Dims& d = plan->dims;
+  info->N = d.N;
+  info->n_blocks = d.nblk;
+  info->q_slots = d.q_slots;
+  info->kv_slots = d.k_slots;
+  info->k_out_max = d.k_out_max;
+  info->q_rows_alloc = d.q_rows_alloc;
+  info->ws_q_tilde = (int64_t)plan->ws.q_tilde;
+  info->ws_k_tilde = (int64_t)plan->ws.k_tilde;
+  info->ws_v_tilde = (int64_t)plan->ws.v_tilde;
+  info->ws_o_tilde = (int64_t)plan->ws.o_tilde;
+  info->ws_n_out = (int64_t)plan->ws.n_out;
+  info->ws_out_base = (int64_t)plan->ws.out_base;
+  info->workspace_bytes = (int64_t)plan->ws.total;
+  return HTTM_OK;
+}
+
+httm_status httm_forward(httm_plan_t plan, const void* Q, const void* K, const void* V, void* out, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  return forward_impl(plan, Q, K, V, out, workspace, workspace_bytes, nullptr, nullptr, stream);
+}
+
+httm_status httm_forward_debug(httm_plan_t plan, const void* Q, const void* K, const void* V, void* out,
+                               void* workspace, size_t workspace_bytes, const httm_debug* dbg, void* stream) {
+  if (!dbg) return HTTM_ERR_ARG;
+  return forward_impl(plan, Q, K, V, out, workspace, workspace_bytes, nullptr, dbg, stream);
+}
+
+httm_status httm_forward_with_plan(httm_plan_t plan, const void* Q, const void* K, const void* V, void* out,
+                                   void* workspace, size_t workspace_bytes, const httm_merge_plan* injected,
+                                   const httm_debug* dbg, void* stream) {
+  if (!injected) return HTTM_ERR_ARG;
+  return forward_impl(plan, Q, K, V, out, workspace, workspace_bytes, injected, dbg, stream);
+}
+
+httm_status httm_reorder(httm_plan_t plan, const void* X, void* Xb, int inverse, void* stream) {
+  if (!plan || !X || !Xb) return HTTM_ERR_ARG;
+  if (plan->dims.mode == HTTM_DENSE) return HTTM_ERR_ARG;
+  if (!aligned16(X) || !aligned16(Xb)) return HTTM_ERR_ALIGN;
+  httm_status st = check_device(plan);
+  if (st != HTTM_OK) return st;
+  cudaError_t e = launch_reorder(plan->dims, plan->fp32, plan->blocks_d, X, Xb, inverse != 0,
+                                 static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? HTTM_OK : HTTM_ERR_CUDA;
+}
+
+httm_status httm_get_device_status(httm_plan_t plan, void* workspace, void* stream, uint32_t* status) {
+  if (!plan || !workspace || !status) return HTTM_ERR_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return HTTM_ERR_CUDA;
+  DevState* st = reinterpret_cast<DevState*>(static_cast<char*>(workspace) + plan->ws.state);
+  uint32_t v = 0;
+  if (cudaMemcpy(&v, &st->status, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return HTTM_ERR_CUDA;
+  if (v && cudaMemset(&st->status, 0, 4) != cudaSuccess) return HTTM_ERR_CUDA;
+  *status = v;
+  if (v & HTTM_DEV_TIMEOUT) return HTTM_ERR_TIMEOUT;
+  if (v) return HTTM_ERR_DEVICE_BOUNDS;
+  return HTTM_OK;
+}
+
+int32_t httm_forward_launches(httm_plan_t plan) { return plan ? plan->launches : -1; }
+
+httm_status httm_profile_enable(httm_plan_t plan, int enable) {
+  if (!plan) return HTTM_ERR_ARG;
+  plan->profile = enable != 0;
+  return HTTM_OK;
+}
+
+httm_status httm_profile_read(httm_plan_t plan, float* ms, int32_t* launches) {
+  if (!plan) return HTTM_ERR_ARG;
+  if (ms)
+    for (int i = 0; i < HTTM_NUM_STAGES; ++i) ms[i] = 0.f;
+  if (launches)
+    for (int i = 0; i < HTTM_NUM_STAGES; ++i) launches[i] = 0;
+  httm_status st = HTTM_OK;
+  for (auto& r : plan->recs) {
+    float t = 0.f;
+    if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess)
+      st = HTTM_ERR_CUDA;
+    if (ms) ms[r.stage] += t;
+    if (launches) launches[r.stage] += r.n;
+    plan->pool.push_back(r.a);
+    plan->pool.push_back(r.b);
+  }
+  plan->recs.clear();
+  return st;
+}
+
+}  // extern "C"

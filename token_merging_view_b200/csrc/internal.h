@@ -1,0 +1,84 @@
+// Internal structures shared by the host planner and the kernels.
+//
+// Token n = t * P + p of head hh lives at row hh * N + n of a [h, N, d]
+// tensor.  Merge blocks follow key design 2 of the HTTM note ("temporal
+// reordering + in-block merging"): block b covers the patches
+// [p0, p0 + s) of frames [t0, t0 + t_g); in-block index i = tau * s + sigma
+// maps to token base + tau * P + sigma with base = t0 * P + p0.  The
+// contiguous variant is one frame-less run: s = n_b, t_g = 1.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+
+namespace httm {
+
+struct BlockDesc {
+  int32_t base;        // original index of in-block token 0
+  int32_t s;           // tokens per frame slice (s_j), n_b for contiguous blocks
+  int32_t n_b;         // tokens in the block
+  int32_t tok_off;     // offset of the block in block order (sum of earlier n_b)
+  int32_t q_ndst, q_r, q_src_off, q_slot_off;   // query plan: dsts, merged, offsets
+  int32_t k_ndst, k_r, k_src_off, k_slot_off;   // key plan (values follow it)
+};
+
+// Everything a kernel needs to know about the layer; passed by value.
+struct Dims {
+  int32_t h, N, P, d;
+  int32_t mode;                  // httm_mode
+  int32_t n_s, n_t, R, contig;   // token -> block mapping
+  int32_t nblk;
+  int32_t q_stride, kv_stride;
+  int32_t q_src, k_src;          // sources per head, all blocks
+  int32_t q_slots, k_slots;      // regular query slots / key-value slots per head
+  int32_t max_ndst, max_nsrc, max_nb;
+  int64_t k_out_max;
+  int64_t out_base;              // first row of the outlier region in Q~ / O~
+  int64_t q_rows_alloc;
+  int32_t nchunk_per_head;       // chunks of the outlier scan per head
+  int32_t max_items;             // attention work items (upper bound)
+  float scale;
+};
+
+constexpr int kChunk = 4096;       // keys per chunk of the outlier compaction
+constexpr int kHistBins = 2048;    // radix digit of the outlier select (11 bits)
+constexpr int kAttnRows = 128;     // query rows per attention work item
+
+// Device-side state at the head of the workspace.
+struct DevState {
+  uint32_t status;               // HTTM_DEV_* bits (sticky until read)
+  uint32_t n_eligible;           // queries in groups of >= 2 tokens
+  uint32_t n_items;              // live attention work items
+  uint32_t pad0;
+  uint32_t sel[8];               // outlier select: threshold key, eq budget, total
+};
+
+struct Workspace {
+  size_t state, hist, chunk, n_out, out_base, items;
+  size_t q_best, q_score, q_merged, k_best, k_score, k_merged;
+  size_t q_slot, keys, mask, q_members, q_gstart, q_gcount;
+  size_t q_tilde, k_tilde, v_tilde, o_tilde;
+  size_t total;
+};
+
+struct Debug;  // mirrors httm_debug
+
+// Pointers into one forward's workspace, resolved on the host.
+struct Buffers {
+  DevState* state;
+  uint32_t* hist;          // [3][kHistBins]
+  uint32_t* chunk;         // [nchunk][4]: gt, eq, take, out_before
+  int32_t* n_out;          // [h]
+  int32_t* out_base;       // [h]
+  int4* items;             // [max_items]: head, q_row0, n_rows, unused
+  int32_t* q_best; float* q_score; uint8_t* q_merged;
+  int32_t* k_best; float* k_score; uint8_t* k_merged;
+  int32_t* q_slot;         // [h, N]
+  uint32_t* keys;          // [h, N]: eligible ? bits(dev) + 1 : 0
+  uint8_t* mask;           // [h, N]
+  int32_t* q_members;      // [h, N]: tokens in group order, per block
+  int32_t* q_gstart;       // [h, q_slots]: first member position (dst groups)
+  int32_t* q_gcount;       // [h, q_slots]
+  void* q_tilde; void* k_tilde; void* v_tilde; void* o_tilde;
+};
+
+}  // namespace httm

@@ -1,0 +1,65 @@
+// Host-side launchers of the kernels (internal; the public ABI is httm.h).
+#pragma once
+#include <cuda_runtime.h>
+
+#include "internal.h"
+
+namespace httm {
+
+// Debug export destinations (device pointers, any may be null).
+struct Debug {
+  int32_t* q_best; float* q_score; uint8_t* q_merged;
+  int32_t* k_best; float* k_score; uint8_t* k_merged;
+  int32_t* q_slot; int32_t* k_slot;
+  float* dev; uint8_t* outlier;
+  float* q_means; float* q_restored; float* k_means; float* v_means;
+};
+
+struct Inject {
+  const int32_t* q_best; const uint8_t* q_merged;
+  const int32_t* k_best; const uint8_t* k_merged;
+  const uint8_t* outlier;
+};
+
+cudaError_t launch_zero_state(const Dims& dims, const Buffers& buf, cudaStream_t s);
+
+cudaError_t launch_match_simt(const Dims& dims, bool fp32, const BlockDesc* blocks,
+                              const int4* items, int n_items, const void* Q, const void* K,
+                              const Buffers& buf, cudaStream_t s);
+
+// Tensor-core matching (bf16, d = 64, head-wise plans).  Returns
+// cudaErrorNotSupported when the shape is not covered.
+cudaError_t launch_match_tc(const Dims& dims, const BlockDesc* blocks, const int4* items,
+                            int n_items, const void* Q, const void* K, const Buffers& buf,
+                            cudaStream_t s);
+
+cudaError_t launch_import_plan(const Dims& dims, const BlockDesc* blocks, const Inject& inj,
+                               const Buffers& buf, cudaStream_t s);
+
+cudaError_t launch_merge(const Dims& dims, bool fp32, const BlockDesc* blocks, bool is_q,
+                         bool injected, const void* X, const void* V, const Buffers& buf,
+                         const Debug& dbg, cudaStream_t s);
+
+cudaError_t launch_outlier(const Dims& dims, bool fp32, const void* Q, bool mask_injected,
+                           const Buffers& buf, cudaStream_t s);
+
+cudaError_t launch_restore(const Dims& dims, bool fp32, const BlockDesc* blocks, const void* Q,
+                           const Buffers& buf, const Debug& dbg, cudaStream_t s);
+
+cudaError_t launch_dense_items(const Dims& dims, const Buffers& buf, cudaStream_t s);
+
+// softmax(Q K^T * scale) V over the work items in buf.items.  q/o rows are
+// indexed by the items; head hh's keys/values are rows [hh * Lk, hh * Lk + Lk).
+cudaError_t launch_attention(const Dims& dims, bool fp32, const void* q, const void* k,
+                             const void* v, void* o, int Lk, const Buffers& buf, cudaStream_t s);
+
+cudaError_t launch_unmerge(const Dims& dims, bool fp32, const Buffers& buf, void* out,
+                           cudaStream_t s);
+
+cudaError_t launch_reorder(const Dims& dims, bool fp32, const BlockDesc* blocks, const void* X,
+                           void* Xb, bool inverse, cudaStream_t s);
+
+cudaError_t launch_export(const Dims& dims, const BlockDesc* blocks, const Buffers& buf,
+                          const Debug& dbg, cudaStream_t s);
+
+}  // namespace httm

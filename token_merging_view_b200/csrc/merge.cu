@@ -1,0 +1,487 @@
+// Top-r mean merging inside a block, the query deviation, the restore step
+// of the outlier filter, and plan import/export.
+//
+// "HTTM: Head-wise Temporal Token Merging for Faster VGGT":
+//  key design 1 -- the top-r sources by match score merge into their best
+//    destination; a merged token is the mean of its members; Q and K merge
+//    independently and V follows K's plan;
+//  key design 3 -- each query's L2 deviation from its merged token (0 if it
+//    was not merged) feeds a global top-d% filter; each outlier is
+//    subtracted from its merged token and kept as a token of its own.
+//
+// One CTA per (block, head).  The top-r choice is a bitonic sort of
+// (~order(score), source ordinal), so ties go to the lower in-block index;
+// the groups come from a second sort of (best destination, source ordinal),
+// which lists every group's members in ascending order.  Sums accumulate in
+// fp32 in member order (destination first), so results are bit-reproducible.
+#include <algorithm>
+
+#include "common.cuh"
+#include "launch.h"
+
+namespace httm {
+namespace {
+
+constexpr int kMergeThreads = 512;
+
+// A [D]-row spread over one warp: lane l owns elements [l*E, l*E + E).
+template <class T, int D>
+struct WarpRow {
+  static constexpr int E = D >= 32 ? D / 32 : 1;
+  __device__ static bool owns(int lane) { return lane * E < D; }
+  __device__ static void load(const T* row, int lane, float (&v)[E]) {
+#pragma unroll
+    for (int e = 0; e < E; ++e) v[e] = owns(lane) ? to_f(row[lane * E + e]) : 0.f;
+  }
+  __device__ static void store(T* row, int lane, const float (&v)[E]) {
+    if (!owns(lane)) return;
+#pragma unroll
+    for (int e = 0; e < E; ++e) row[lane * E + e] = from_f<T>(v[e]);
+  }
+};
+
+template <>
+struct WarpRow<__nv_bfloat16, 64> {
+  static constexpr int E = 2;
+  __device__ static bool owns(int) { return true; }
+  __device__ static void load(const __nv_bfloat16* row, int lane, float (&v)[2]) {
+    const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(row) + lane);
+    v[0] = __uint_as_float(w << 16);
+    v[1] = __uint_as_float(w & 0xffff0000u);
+  }
+  __device__ static void store(__nv_bfloat16* row, int lane, const float (&v)[2]) {
+    reinterpret_cast<__nv_bfloat162*>(row)[lane] = __floats2bfloat162_rn(v[0], v[1]);
+  }
+};
+
+template <int E>
+__device__ __forceinline__ void store_f32(float* row, int lane, int D, const float (&v)[E]) {
+#pragma unroll
+  for (int e = 0; e < E; ++e)
+    if (lane * E + e < D) row[lane * E + e] = v[e];
+}
+
+// Exclusive scan of in[0, n) into out[0, n) by the whole block.
+__device__ void block_scan_array(const int32_t* in, int32_t* out, int n, uint32_t* tmp) {
+  const int per = (n + blockDim.x - 1) / blockDim.x;
+  const int lo = min(n, (int)threadIdx.x * per), hi = min(n, lo + per);
+  uint32_t s = 0;
+  for (int i = lo; i < hi; ++i) s += in[i];
+  uint32_t tot;
+  uint32_t run = block_excl_scan(s, tmp, &tot);
+  for (int i = lo; i < hi; ++i) {
+    out[i] = run;
+    run += in[i];
+  }
+  __syncthreads();
+}
+
+template <class T, int D, bool IS_Q>
+__global__ void __launch_bounds__(kMergeThreads)
+merge_kernel(Dims dims, const BlockDesc* __restrict__ blocks, const T* __restrict__ X,
+             const T* __restrict__ V, Buffers buf, Debug dbg, int injected, int sortN) {
+  using Row = WarpRow<T, D>;
+  constexpr int E = Row::E;
+  extern __shared__ __align__(16) unsigned char smem[];
+  unsigned long long* keys = reinterpret_cast<unsigned long long*>(smem);
+  int32_t* cnt = reinterpret_cast<int32_t*>(keys + sortN);
+  int32_t* gst = cnt + dims.max_ndst;
+  uint32_t* hist = reinterpret_cast<uint32_t*>(gst + dims.max_ndst);
+  uint32_t* tmp = hist + (IS_Q ? kHistBins : 0);
+  __shared__ int s_bad;
+  __shared__ uint32_t s_elig;
+
+  const int tid = threadIdx.x, bd = blockDim.x;
+  const int lane = tid & 31, warp = tid >> 5, nwarps = bd >> 5;
+  const int hh = blockIdx.y;
+  const BlockDesc b = blocks[blockIdx.x];
+  const int stride = IS_Q ? dims.q_stride : dims.kv_stride;
+  const int ndst = IS_Q ? b.q_ndst : b.k_ndst;
+  const int r = IS_Q ? b.q_r : b.k_r;
+  const int nsrc = b.n_b - ndst;
+  const size_t sbase = (size_t)hh * (IS_Q ? dims.q_src : dims.k_src) + (IS_Q ? b.q_src_off : b.k_src_off);
+  const int32_t* best = (IS_Q ? buf.q_best : buf.k_best) + sbase;
+  const float* score = (IS_Q ? buf.q_score : buf.k_score) + sbase;
+  uint8_t* merged = (IS_Q ? buf.q_merged : buf.k_merged) + sbase;
+  const int slot_off = IS_Q ? b.q_slot_off : b.k_slot_off;
+  const int nslots = IS_Q ? dims.q_slots : dims.k_slots;
+  const size_t tokbase = (size_t)hh * dims.N;
+
+  if (cta_plan_failed(buf.state)) return;
+  if (tid == 0) { s_bad = 0; s_elig = 0; }
+  if (IS_Q)
+    for (int i = tid; i < kHistBins; i += bd) hist[i] = 0;
+
+  // 1. top-r: the r sources with the largest (score, -ordinal) merge.
+  if (!injected) {
+    for (int k = tid; k < sortN; k += bd)
+      keys[k] = k < nsrc ? ((unsigned long long)(~float_order(score[k])) << 32) | (unsigned)k : ~0ull;
+    __syncthreads();
+    block_bitonic_sort(keys, sortN);
+    for (int p = tid; p < nsrc; p += bd) merged[(uint32_t)keys[p]] = p < r ? 1 : 0;
+    __syncthreads();
+  } else {
+    uint32_t c = 0;
+    for (int k = tid; k < nsrc; k += bd) c += merged[k] != 0;
+    uint32_t tot;
+    block_excl_scan(c, tmp, &tot);
+    if (tid == 0 && tot != (uint32_t)r) s_bad = 1;
+  }
+
+  // 2. group members: (best destination, ordinal) for merged sources, kept
+  //    sources after them in ascending ordinal.
+  for (int k = tid; k < sortN; k += bd) {
+    unsigned long long v = ~0ull;
+    if (k < nsrc) {
+      if (merged[k]) {
+        int m = best[k];
+        if (m < 0 || m >= ndst) { s_bad = 1; m = 0; }
+        v = ((unsigned long long)m << 32) | (unsigned)k;
+      } else {
+        v = (0xFFFFFFFFull << 32) | (unsigned)k;
+      }
+    }
+    keys[k] = v;
+  }
+  for (int m = tid; m < ndst; m += bd) cnt[m] = 1;
+  __syncthreads();
+  if (s_bad) {
+    if (tid == 0) set_status(buf.state, HTTM_DEV_BAD_PLAN);
+    return;
+  }
+  block_bitonic_sort(keys, sortN);
+  for (int p = tid; p < r; p += bd) atomicAdd(&cnt[keys[p] >> 32], 1);
+  __syncthreads();
+  block_scan_array(cnt, gst, ndst, tmp);
+
+  const T* Xh = X + tokbase * D;
+  const T* Vh = IS_Q ? nullptr : V + tokbase * D;
+  T* Xt = reinterpret_cast<T*>(IS_Q ? buf.q_tilde : buf.k_tilde) + (size_t)hh * nslots * D;
+  T* Vt = IS_Q ? nullptr : reinterpret_cast<T*>(buf.v_tilde) + (size_t)hh * nslots * D;
+  float* dmean = IS_Q ? dbg.q_means : dbg.k_means;
+  uint32_t elig = 0;
+
+  // 3. destination groups: mean of members; queries also get deviations.
+  for (int m = warp; m < ndst; m += nwarps) {
+    const int c = cnt[m];
+    const int ms = gst[m] - m;  // first merged member in keys[]
+    const int slot = slot_off + m;
+    float acc[E], accv[E], x[E];
+    const int tok0 = block_token(b, m * stride, dims.P);
+    Row::load(Xh + (size_t)tok0 * D, lane, acc);
+    if (!IS_Q) Row::load(Vh + (size_t)tok0 * D, lane, accv);
+    for (int q = 0; q < c - 1; ++q) {
+      const int tok = block_token(b, src_index((int)(uint32_t)keys[ms + q], stride), dims.P);
+      Row::load(Xh + (size_t)tok * D, lane, x);
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc[e] += x[e];
+      if (!IS_Q) {
+        Row::load(Vh + (size_t)tok * D, lane, x);
+#pragma unroll
+        for (int e = 0; e < E; ++e) accv[e] += x[e];
+      }
+    }
+    const float fc = (float)c;
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc[e] = acc[e] / fc;
+    Row::store(Xt + (size_t)slot * D, lane, acc);
+    if (dmean) store_f32<E>(dmean + ((size_t)hh * nslots + slot) * D, lane, D, acc);
+    if (!IS_Q) {
+#pragma unroll
+      for (int e = 0; e < E; ++e) accv[e] = accv[e] / fc;
+      Row::store(Vt + (size_t)slot * D, lane, accv);
+      if (dbg.v_means) store_f32<E>(dbg.v_means + ((size_t)hh * nslots + slot) * D, lane, D, accv);
+    }
+    const int pos = b.tok_off + gst[m];
+    if (IS_Q && lane == 0) {
+      buf.q_gstart[(size_t)hh * nslots + slot] = pos;
+      buf.q_gcount[(size_t)hh * nslots + slot] = c;
+    }
+    for (int q = 0; q < c; ++q) {
+      const int tok = q == 0 ? tok0
+                             : block_token(b, src_index((int)(uint32_t)keys[ms + q - 1], stride), dims.P);
+      if (IS_Q) {
+        uint32_t key = 0;
+        if (c >= 2) {
+          Row::load(Xh + (size_t)tok * D, lane, x);
+          float ss = 0.f;
+#pragma unroll
+          for (int e = 0; e < E; ++e) {
+            const float df = x[e] - acc[e];
+            ss = fmaf(df, df, ss);
+          }
+          ss = warp_sum(ss);
+          key = __float_as_uint(sqrtf(ss)) + 1u;
+        }
+        if (lane == 0) {
+          buf.q_members[tokbase + pos + q] = tok;
+          buf.q_slot[tokbase + tok] = slot;
+          buf.keys[tokbase + tok] = key;
+          if (key) {
+            atomicAdd(&hist[key >> 21], 1u);
+            ++elig;
+          }
+        }
+      } else if (dbg.k_slot && lane == 0) {
+        dbg.k_slot[tokbase + tok] = slot;
+      }
+    }
+  }
+
+  // 4. kept sources: singleton slots after the destination groups.
+  for (int p = r + warp; p < nsrc; p += nwarps) {
+    const int rank = p - r;
+    const int slot = slot_off + ndst + rank;
+    const int tok = block_token(b, src_index((int)(uint32_t)keys[p], stride), dims.P);
+    float x[E];
+    Row::load(Xh + (size_t)tok * D, lane, x);
+    Row::store(Xt + (size_t)slot * D, lane, x);
+    if (dmean) store_f32<E>(dmean + ((size_t)hh * nslots + slot) * D, lane, D, x);
+    if (!IS_Q) {
+      Row::load(Vh + (size_t)tok * D, lane, x);
+      Row::store(Vt + (size_t)slot * D, lane, x);
+      if (dbg.v_means) store_f32<E>(dbg.v_means + ((size_t)hh * nslots + slot) * D, lane, D, x);
+      if (dbg.k_slot && lane == 0) dbg.k_slot[tokbase + tok] = slot;
+    } else if (lane == 0) {
+      const int pos = b.tok_off + ndst + r + rank;
+      buf.q_members[tokbase + pos] = tok;
+      buf.q_slot[tokbase + tok] = slot;
+      buf.keys[tokbase + tok] = 0u;
+      buf.q_gstart[(size_t)hh * nslots + slot] = pos;
+      buf.q_gcount[(size_t)hh * nslots + slot] = 1;
+    }
+  }
+
+  if (IS_Q) {
+    if (lane == 0 && elig) atomicAdd(&s_elig, elig);
+    __syncthreads();
+    for (int i = tid; i < kHistBins; i += bd)
+      if (hist[i]) atomicAdd(&buf.hist[i], hist[i]);
+    if (tid == 0 && s_elig) atomicAdd(&buf.state->n_eligible, s_elig);
+  }
+}
+
+// Restore (key design 3): every regular query slot holding outliers becomes
+// the mean of its remaining members; a slot whose members are all outliers
+// is drained (zeros; no token reads it).
+template <class T, int D>
+__global__ void __launch_bounds__(256)
+restore_kernel(Dims dims, const BlockDesc* __restrict__ blocks, const T* __restrict__ Q, Buffers buf,
+               Debug dbg) {
+  using Row = WarpRow<T, D>;
+  constexpr int E = Row::E;
+  if (plan_failed(buf.state)) return;
+  if (buf.state->sel[3] == 0 && dbg.q_restored == nullptr) return;  // no outlier anywhere
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  const int hh = blockIdx.y;
+  const BlockDesc b = blocks[blockIdx.x];
+  const size_t tokbase = (size_t)hh * dims.N;
+  const T* Qh = Q + tokbase * D;
+  T* Qt = reinterpret_cast<T*>(buf.q_tilde) + (size_t)hh * dims.q_slots * D;
+  const int nslot_b = b.n_b - b.q_r;
+  for (int s = warp; s < nslot_b; s += nwarps) {
+    const int slot = b.q_slot_off + s;
+    const int gs = buf.q_gstart[(size_t)hh * dims.q_slots + slot];
+    const int gc = buf.q_gcount[(size_t)hh * dims.q_slots + slot];
+    if (gc < 2 && dbg.q_restored == nullptr) continue;
+    if (gs < 0 || gc < 1 || gs + gc > dims.N) {
+      if (lane == 0) set_status(buf.state, HTTM_DEV_BOUNDS);
+      continue;
+    }
+    int nout = 0;
+    for (int q = lane; q < gc; q += 32) {
+      const int tok = buf.q_members[tokbase + gs + q];
+      if (tok < 0 || tok >= dims.N) {
+        set_status(buf.state, HTTM_DEV_BOUNDS);
+        continue;
+      }
+      nout += buf.mask[tokbase + tok] != 0;
+    }
+    nout = __reduce_add_sync(0xffffffffu, nout);
+    if (nout == 0 && dbg.q_restored == nullptr) continue;
+    float acc[E], x[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc[e] = 0.f;
+    for (int q = 0; q < gc; ++q) {
+      const int tok = buf.q_members[tokbase + gs + q];
+      if (tok < 0 || tok >= dims.N || buf.mask[tokbase + tok]) continue;
+      Row::load(Qh + (size_t)tok * D, lane, x);
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc[e] += x[e];
+    }
+    const int remain = gc - nout;
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc[e] = remain ? acc[e] / (float)remain : 0.f;
+    if (nout > 0) Row::store(Qt + (size_t)slot * D, lane, acc);
+    if (dbg.q_restored) {
+      float o[E];
+#pragma unroll
+      for (int e = 0; e < E; ++e) o[e] = remain ? acc[e] : __int_as_float(0x7fc00000);
+      store_f32<E>(dbg.q_restored + ((size_t)hh * dims.q_slots + slot) * D, lane, D, o);
+    }
+  }
+}
+
+// Injected plan -> internal source-order arrays, with validation.
+__global__ void import_kernel(Dims dims, const BlockDesc* __restrict__ blocks, Inject inj, Buffers buf) {
+  const size_t total = 2ull * dims.h * dims.N;
+  for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < total;
+       idx += (size_t)gridDim.x * blockDim.x) {
+    const int tensor = (int)(idx / ((size_t)dims.h * dims.N));
+    const size_t rem = idx - (size_t)tensor * dims.h * dims.N;
+    const int hh = (int)(rem / dims.N);
+    const int n = (int)(rem - (size_t)hh * dims.N);
+    if (tensor == 0 && inj.outlier) buf.mask[rem] = inj.outlier[rem] ? 1 : 0;
+    if (inj.q_best == nullptr) continue;
+    const int stride = tensor == 0 ? dims.q_stride : dims.kv_stride;
+    int blk, i;
+    token_block(dims, n, blk, i);
+    if (i % stride == 0) continue;
+    const BlockDesc b = blocks[blk];
+    const int k = src_ordinal(i, stride);
+    const int32_t* ib = tensor == 0 ? inj.q_best : inj.k_best;
+    const uint8_t* im = tensor == 0 ? inj.q_merged : inj.k_merged;
+    const int nd = ib[rem];
+    int m = 0;
+    const bool mg = im[rem] != 0;
+    if (mg) {
+      bool ok = nd >= 0 && nd < dims.N;
+      if (ok) {
+        int blk2, i2;
+        token_block(dims, nd, blk2, i2);
+        ok = blk2 == blk && i2 % stride == 0;
+        if (ok) m = i2 / stride;
+      }
+      if (!ok) set_status(buf.state, HTTM_DEV_BAD_PLAN);
+    }
+    const size_t si = (size_t)hh * (tensor == 0 ? dims.q_src : dims.k_src) +
+                      (tensor == 0 ? b.q_src_off : b.k_src_off) + k;
+    (tensor == 0 ? buf.q_best : buf.k_best)[si] = m;
+    (tensor == 0 ? buf.q_merged : buf.k_merged)[si] = mg ? 1 : 0;
+    (tensor == 0 ? buf.q_score : buf.k_score)[si] = 0.f;
+  }
+}
+
+// Internal arrays -> the [h, N] original-order debug exports.
+__global__ void export_kernel(Dims dims, const BlockDesc* __restrict__ blocks, Buffers buf, Debug dbg) {
+  if (plan_failed(buf.state)) return;
+  const size_t total = (size_t)dims.h * dims.N;
+  for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < total;
+       idx += (size_t)gridDim.x * blockDim.x) {
+    const int hh = (int)(idx / dims.N);
+    const int n = (int)(idx - (size_t)hh * dims.N);
+    int blk, i;
+    token_block(dims, n, blk, i);
+    const BlockDesc b = blocks[blk];
+#pragma unroll
+    for (int tensor = 0; tensor < 2; ++tensor) {
+      int32_t* ob = tensor == 0 ? dbg.q_best : dbg.k_best;
+      float* os = tensor == 0 ? dbg.q_score : dbg.k_score;
+      uint8_t* om = tensor == 0 ? dbg.q_merged : dbg.k_merged;
+      if (!ob && !os && !om) continue;
+      const int stride = tensor == 0 ? dims.q_stride : dims.kv_stride;
+      int bt = -1, mg = 0;
+      float sc = 0.f;
+      if (i % stride != 0) {
+        const size_t si = (size_t)hh * (tensor == 0 ? dims.q_src : dims.k_src) +
+                          (tensor == 0 ? b.q_src_off : b.k_src_off) + src_ordinal(i, stride);
+        bt = block_token(b, (tensor == 0 ? buf.q_best : buf.k_best)[si] * stride, dims.P);
+        sc = (tensor == 0 ? buf.q_score : buf.k_score)[si];
+        mg = (tensor == 0 ? buf.q_merged : buf.k_merged)[si];
+      }
+      if (ob) ob[idx] = bt;
+      if (os) os[idx] = sc;
+      if (om) om[idx] = (uint8_t)mg;
+    }
+    if (dbg.q_slot) dbg.q_slot[idx] = buf.q_slot[idx];
+    if (dbg.dev) {
+      const uint32_t key = buf.keys[idx];
+      dbg.dev[idx] = key ? __uint_as_float(key - 1u) : 0.f;
+    }
+    if (dbg.outlier) dbg.outlier[idx] = buf.mask[idx];
+  }
+}
+
+__global__ void zero_state_kernel(Buffers buf) {
+  for (int i = threadIdx.x; i < 3 * kHistBins; i += blockDim.x) buf.hist[i] = 0u;
+  if (threadIdx.x == 0) {
+    buf.state->status = 0u;
+    buf.state->n_eligible = 0u;
+    buf.state->n_items = 0u;
+  }
+  if (threadIdx.x < 8) buf.state->sel[threadIdx.x] = 0u;
+}
+
+int next_pow2(int x) {
+  int p = 32;
+  while (p < x) p <<= 1;
+  return p;
+}
+
+template <class T, int D>
+cudaError_t launch_merge_t(const Dims& dims, const BlockDesc* blocks, bool is_q, bool injected,
+                           const void* X, const void* V, const Buffers& buf, const Debug& dbg,
+                           cudaStream_t s) {
+  const int sortN = next_pow2(dims.max_nsrc);
+  const size_t smem = (size_t)sortN * 8 + 2ull * dims.max_ndst * 4 + (is_q ? kHistBins * 4 : 0) + 64 * 4;
+  dim3 grid(dims.nblk, dims.h);
+  if (is_q) {
+    auto k = merge_kernel<T, D, true>;
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    k<<<grid, kMergeThreads, smem, s>>>(dims, blocks, (const T*)X, nullptr, buf, dbg, injected, sortN);
+  } else {
+    auto k = merge_kernel<T, D, false>;
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    k<<<grid, kMergeThreads, smem, s>>>(dims, blocks, (const T*)X, (const T*)V, buf, dbg, injected, sortN);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_zero_state(const Dims&, const Buffers& buf, cudaStream_t s) {
+  zero_state_kernel<<<1, 1024, 0, s>>>(buf);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_merge(const Dims& dims, bool fp32, const BlockDesc* blocks, bool is_q, bool injected,
+                         const void* X, const void* V, const Buffers& buf, const Debug& dbg,
+                         cudaStream_t s) {
+  if (fp32) {
+    if (dims.d == 16) return launch_merge_t<float, 16>(dims, blocks, is_q, injected, X, V, buf, dbg, s);
+    return launch_merge_t<float, 64>(dims, blocks, is_q, injected, X, V, buf, dbg, s);
+  }
+  if (dims.d == 16) return launch_merge_t<__nv_bfloat16, 16>(dims, blocks, is_q, injected, X, V, buf, dbg, s);
+  return launch_merge_t<__nv_bfloat16, 64>(dims, blocks, is_q, injected, X, V, buf, dbg, s);
+}
+
+cudaError_t launch_restore(const Dims& dims, bool fp32, const BlockDesc* blocks, const void* Q,
+                           const Buffers& buf, const Debug& dbg, cudaStream_t s) {
+  dim3 grid(dims.nblk, dims.h);
+  if (fp32) {
+    if (dims.d == 16) restore_kernel<float, 16><<<grid, 256, 0, s>>>(dims, blocks, (const float*)Q, buf, dbg);
+    else restore_kernel<float, 64><<<grid, 256, 0, s>>>(dims, blocks, (const float*)Q, buf, dbg);
+  } else {
+    if (dims.d == 16) restore_kernel<__nv_bfloat16, 16><<<grid, 256, 0, s>>>(dims, blocks, (const __nv_bfloat16*)Q, buf, dbg);
+    else restore_kernel<__nv_bfloat16, 64><<<grid, 256, 0, s>>>(dims, blocks, (const __nv_bfloat16*)Q, buf, dbg);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_import_plan(const Dims& dims, const BlockDesc* blocks, const Inject& inj,
+                               const Buffers& buf, cudaStream_t s) {
+  const size_t total = 2ull * dims.h * dims.N;
+  const int grid = (int)std::min<size_t>((total + 255) / 256, 148 * 16);
+  import_kernel<<<grid, 256, 0, s>>>(dims, blocks, inj, buf);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_export(const Dims& dims, const BlockDesc* blocks, const Buffers& buf, const Debug& dbg,
+                          cudaStream_t s) {
+  const size_t total = (size_t)dims.h * dims.N;
+  const int grid = (int)std::min<size_t>((total + 255) / 256, 148 * 16);
+  export_kernel<<<grid, 256, 0, s>>>(dims, blocks, buf, dbg);
+  return cudaGetLastError();
+}
+
+}  // namespace httm

@@ -1,0 +1,318 @@
+// Cross-head adaptive outlier filter, the global selection part.
+//
+// "HTTM: Head-wise Temporal Token Merging for Faster VGGT", key design 3:
+// the deviations of all heads' queries compete for one budget: the top-d%
+// form the mask M_o in {0,1}^{h x N}.  Here the budget is
+// k = min(floor(d% * h * N / 100), #eligible) and the order is
+// (deviation desc, flat index h * N + n asc).
+//
+// Each query carries a 32-bit key = bits(dev) + 1 if it sits in a group of
+// >= 2 tokens, else 0 (dev >= 0, so float bits order like the values).  The
+// k-th largest key T is found by a three-digit radix select (11 + 11 + 10
+// bits); the first digit's histogram is built by the query merge kernel.
+// Then keys > T are outliers, plus the first (k - #{key > T}) keys equal to
+// T in flat-index order, found with chunk counts and a scan.  Every step is
+// its own launch (no grid-wide barrier, no spin wait), and every count is an
+// integer, so the mask is deterministic.
+#include <algorithm>
+
+#include "common.cuh"
+#include "launch.h"
+
+namespace httm {
+namespace {
+
+__device__ __forceinline__ uint32_t k_total(const Dims& dims, const Buffers& buf) {
+  const unsigned long long e = buf.state->n_eligible;
+  return (uint32_t)min((unsigned long long)dims.k_out_max, e);
+}
+
+// One full warp: the bin holding the k-th largest key (k >= 1) of hist[0, nb)
+// and k minus the number of keys in higher bins.
+__device__ void select_bin(const uint32_t* hist, int nb, uint32_t k, int* bin, uint32_t* krem) {
+  const int lane = threadIdx.x & 31;
+  uint32_t above = 0;
+  for (int top = nb - 1; top >= 0; top -= 32) {
+    const int bb = top - lane;
+    const uint32_t c = bb >= 0 ? hist[bb] : 0u;
+    const uint32_t inc = warp_incl_scan(c);
+    const uint32_t tot = __shfl_sync(0xffffffffu, inc, 31);
+    if (above + tot >= k) {
+      const unsigned ballot = __ballot_sync(0xffffffffu, above + inc >= k);
+      const int l = __ffs(ballot) - 1;
+      const uint32_t inc_l = __shfl_sync(0xffffffffu, inc, l);
+      const uint32_t c_l = __shfl_sync(0xffffffffu, c, l);
+      *bin = top - l;
+      *krem = k - (above + inc_l - c_l);
+      return;
+    }
+    above += tot;
+  }
+  *bin = 0;
+  *krem = 0;
+}
+
+// Selected digits of the passes done so far (computed by warp 0 of each CTA).
+struct Sel {
+  int b1, b2, b3;
+  uint32_t k1, k2, k3;
+};
+
+__device__ void select_digits(const Buffers& buf, uint32_t k, int passes, Sel* s) {
+  if ((threadIdx.x >> 5) != 0) return;
+  select_bin(buf.hist, kHistBins, k, &s->b1, &s->k1);
+  if (passes >= 2) select_bin(buf.hist + kHistBins, kHistBins, s->k1, &s->b2, &s->k2);
+  if (passes >= 3) select_bin(buf.hist + 2 * kHistBins, 1024, s->k2, &s->b3, &s->k3);
+}
+
+// Histogram of the next digit among keys whose higher digits were selected.
+__global__ void __launch_bounds__(1024) hist_pass_kernel(Dims dims, Buffers buf, int pass) {
+  __shared__ uint32_t sh[kHistBins];
+  __shared__ Sel sel;
+  if (cta_plan_failed(buf.state)) return;
+  const uint32_t k = k_total(dims, buf);
+  if (k == 0) return;
+  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sh[i] = 0u;
+  select_digits(buf, k, pass - 1, &sel);
+  __syncthreads();
+  const size_t total = (size_t)dims.h * dims.N;
+  const uint32_t pre = pass == 2 ? (uint32_t)sel.b1 : ((uint32_t)sel.b1 << 11) | (uint32_t)sel.b2;
+  const int shift = pass == 2 ? 21 : 10;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
+    const uint32_t key = buf.keys[i];
+    if ((key >> shift) == pre) atomicAdd(&sh[pass == 2 ? (key >> 10) & 2047u : key & 1023u], 1u);
+  }
+  __syncthreads();
+  uint32_t* gh = buf.hist + (pass - 1) * kHistBins;
+  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x)
+    if (sh[i]) atomicAdd(&gh[i], sh[i]);
+}
+
+// Per chunk of kChunk consecutive queries of one head: #{key > T}, #{key == T}.
+__global__ void __launch_bounds__(1024) out_count_kernel(Dims dims, Buffers buf, int mask_injected) {
+  __shared__ Sel sel;
+  __shared__ uint32_t tmp[40];
+  if (cta_plan_failed(buf.state)) return;
+  const int c = blockIdx.x;
+  const int hh = c / dims.nchunk_per_head, cc = c - hh * dims.nchunk_per_head;
+  const int lo = cc * kChunk, hi = min(dims.N, lo + kChunk);
+  const size_t base = (size_t)hh * dims.N;
+  uint32_t gt = 0, eq = 0, T = 0xffffffffu, need = 0;
+  const uint32_t k = k_total(dims, buf);
+  if (!mask_injected) {
+    if (k > 0) {
+      select_digits(buf, k, 3, &sel);
+      __syncthreads();
+      T = ((uint32_t)sel.b1 << 21) | ((uint32_t)sel.b2 << 10) | (uint32_t)sel.b3;
+      need = sel.k3;
+      for (int n = lo + threadIdx.x; n < hi; n += blockDim.x) {
+        const uint32_t key = buf.keys[base + n];
+        gt += key > T;
+        eq += key == T;
+      }
+    }
+  } else {
+    for (int n = lo + threadIdx.x; n < hi; n += blockDim.x) {
+      if (buf.mask[base + n]) {
+        ++gt;
+        if (buf.keys[base + n] == 0u) set_status(buf.state, HTTM_DEV_BAD_PLAN);
+      }
+    }
+  }
+  uint32_t tot;
+  block_excl_scan(gt, tmp, &tot);
+  gt = tot;
+  block_excl_scan(eq, tmp, &tot);
+  eq = tot;
+  if (threadIdx.x == 0) {
+    buf.chunk[4 * c + 0] = gt;
+    buf.chunk[4 * c + 1] = eq;
+    if (c == 0) {
+      buf.state->sel[0] = T;
+      buf.state->sel[1] = need;
+      buf.state->sel[2] = k;
+    }
+  }
+}
+
+// One CTA: which equal keys are taken, outlier offsets per chunk and head,
+// the outlier row ranges, and the attention work list.
+__global__ void __launch_bounds__(1024) out_scan_kernel(Dims dims, Buffers buf) {
+  __shared__ uint32_t tmp[40];
+  __shared__ int tile_off[65];
+  if (cta_plan_failed(buf.state)) return;
+  const int tid = threadIdx.x;
+  const int cph = dims.nchunk_per_head;
+  const int nchunk = dims.h * cph;
+  const uint32_t need = buf.state->sel[1];
+  uint32_t carry = 0;
+  for (int base = 0; base < nchunk; base += blockDim.x) {
+    const int c = base + tid;
+    const uint32_t eq = c < nchunk ? buf.chunk[4 * c + 1] : 0u;
+    uint32_t tot;
+    const uint32_t ex = block_excl_scan(eq, tmp, &tot) + carry;
+    if (c < nchunk) {
+      const uint32_t take = need > ex ? min(need - ex, eq) : 0u;
+      buf.chunk[4 * c + 2] = take;
+      buf.chunk[4 * c + 3] = buf.chunk[4 * c + 0] + take;
+    }
+    carry += tot;
+  }
+  __syncthreads();
+  for (int hh = 0; hh < dims.h; ++hh) {
+    uint32_t run = 0;
+    for (int base = 0; base < cph; base += blockDim.x) {
+      const int c = hh * cph + base + tid;
+      const bool in = base + tid < cph;
+      const uint32_t v = in ? buf.chunk[4 * c + 3] : 0u;
+      uint32_t tot;
+      const uint32_t ex = block_excl_scan(v, tmp, &tot) + run;
+      if (in) buf.chunk[4 * c + 3] = ex;
+      run += tot;
+    }
+    if (tid == 0) buf.n_out[hh] = (int32_t)run;
+    __syncthreads();
+  }
+  if (tid == 0) {
+    unsigned long long total = 0;
+    for (int hh = 0; hh < dims.h; ++hh) total += (uint32_t)buf.n_out[hh];
+    if (total > (unsigned long long)dims.k_out_max) {
+      set_status(buf.state, HTTM_DEV_BAD_PLAN);
+      for (int hh = 0; hh < dims.h; ++hh) buf.n_out[hh] = 0;
+      total = 0;
+    }
+    long long row = dims.out_base;
+    int tiles = 0;
+    for (int hh = 0; hh < dims.h; ++hh) {
+      buf.out_base[hh] = (int32_t)row;
+      row += ((buf.n_out[hh] + kAttnRows - 1) / kAttnRows) * kAttnRows;
+      tile_off[hh] = tiles;
+      tiles += (buf.n_out[hh] + kAttnRows - 1) / kAttnRows;
+    }
+    tile_off[dims.h] = tiles;
+    buf.state->sel[3] = (uint32_t)total;
+  }
+  __syncthreads();
+  const int tq = (dims.q_slots + kAttnRows - 1) / kAttnRows;
+  const int nreg = dims.h * tq;
+  for (int i = tid; i < nreg; i += blockDim.x) {
+    const int hh = i / tq, t = i - hh * tq;
+    buf.items[i] = make_int4(hh, hh * dims.q_slots + t * kAttnRows, min(kAttnRows, dims.q_slots - t * kAttnRows), 0);
+  }
+  for (int hh = 0; hh < dims.h; ++hh) {
+    const int nt = tile_off[hh + 1] - tile_off[hh];
+    for (int t = tid; t < nt; t += blockDim.x)
+      buf.items[nreg + tile_off[hh] + t] =
+          make_int4(hh, buf.out_base[hh] + t * kAttnRows, min(kAttnRows, buf.n_out[hh] - t * kAttnRows), 0);
+  }
+  if (tid == 0) buf.state->n_items = (uint32_t)(nreg + tile_off[dims.h]);
+}
+
+// Per chunk: decide each query, write M_o, give outliers their slots and
+// copy each outlier's own row into its slot of Q~.
+template <class T, int D>
+__global__ void __launch_bounds__(1024)
+out_emit_kernel(Dims dims, const T* __restrict__ Q, Buffers buf, int mask_injected) {
+  __shared__ uint32_t tmp[40];
+  constexpr int PER = kChunk / 1024;
+  if (cta_plan_failed(buf.state)) return;
+  const int c = blockIdx.x;
+  const int hh = c / dims.nchunk_per_head, cc = c - hh * dims.nchunk_per_head;
+  const int lo = cc * kChunk, hi = min(dims.N, lo + kChunk);
+  const size_t base = (size_t)hh * dims.N;
+  const uint32_t total_out = buf.state->sel[3];
+  if (total_out == 0) {
+    for (int n = lo + threadIdx.x; n < hi; n += blockDim.x) buf.mask[base + n] = 0;
+    return;
+  }
+  const uint32_t Tk = buf.state->sel[0];
+  const uint32_t take = buf.chunk[4 * c + 2];
+  const uint32_t obefore = buf.chunk[4 * c + 3];
+  const int n0 = lo + threadIdx.x * PER;
+  bool gt[PER], eq[PER];
+  uint32_t neq = 0;
+#pragma unroll
+  for (int j = 0; j < PER; ++j) {
+    const int n = n0 + j;
+    gt[j] = eq[j] = false;
+    if (n < hi) {
+      if (mask_injected) {
+        gt[j] = buf.mask[base + n] != 0;
+      } else {
+        const uint32_t key = buf.keys[base + n];
+        gt[j] = key > Tk;
+        eq[j] = key == Tk;
+      }
+    }
+    neq += eq[j];
+  }
+  uint32_t tot;
+  uint32_t eq_rank = block_excl_scan(neq, tmp, &tot);
+  bool out[PER];
+  uint32_t nout = 0;
+#pragma unroll
+  for (int j = 0; j < PER; ++j) {
+    out[j] = gt[j] || (eq[j] && eq_rank < take);
+    eq_rank += eq[j];
+    nout += out[j];
+  }
+  uint32_t rank = obefore + block_excl_scan(nout, tmp, &tot);
+  const T* Qh = Q + base * D;
+  T* Qt = reinterpret_cast<T*>(buf.q_tilde);
+#pragma unroll
+  for (int j = 0; j < PER; ++j) {
+    const int n = n0 + j;
+    if (n >= hi) continue;
+    buf.mask[base + n] = out[j] ? 1 : 0;
+    if (out[j]) {
+      buf.q_slot[base + n] = dims.q_slots + (int32_t)rank;
+      const T* src = Qh + (size_t)n * D;
+      T* dst = Qt + ((size_t)buf.out_base[hh] + rank) * D;
+      constexpr int VEC = (int)(D * sizeof(T) / 16);
+#pragma unroll
+      for (int v = 0; v < VEC; ++v)
+        reinterpret_cast<uint4*>(dst)[v] = __ldg(reinterpret_cast<const uint4*>(src) + v);
+      ++rank;
+    }
+  }
+}
+
+__global__ void dense_items_kernel(Dims dims, Buffers buf) {
+  const int tq = (dims.N + kAttnRows - 1) / kAttnRows;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < dims.h * tq; i += gridDim.x * blockDim.x) {
+    const int hh = i / tq, t = i - hh * tq;
+    buf.items[i] = make_int4(hh, hh * dims.N + t * kAttnRows, min(kAttnRows, dims.N - t * kAttnRows), 0);
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0) buf.state->n_items = (uint32_t)(dims.h * tq);
+}
+
+}  // namespace
+
+cudaError_t launch_outlier(const Dims& dims, bool fp32, const void* Q, bool mask_injected,
+                           const Buffers& buf, cudaStream_t s) {
+  const size_t total = (size_t)dims.h * dims.N;
+  const int hgrid = (int)std::max<size_t>(1, std::min<size_t>((total + 4095) / 4096, 148 * 2));
+  if (!mask_injected) {
+    hist_pass_kernel<<<hgrid, 1024, 0, s>>>(dims, buf, 2);
+    hist_pass_kernel<<<hgrid, 1024, 0, s>>>(dims, buf, 3);
+  }
+  const int nchunk = dims.h * dims.nchunk_per_head;
+  out_count_kernel<<<nchunk, 1024, 0, s>>>(dims, buf, mask_injected ? 1 : 0);
+  out_scan_kernel<<<1, 1024, 0, s>>>(dims, buf);
+  const int mi = mask_injected ? 1 : 0;
+  if (fp32) {
+    if (dims.d == 16) out_emit_kernel<float, 16><<<nchunk, 1024, 0, s>>>(dims, (const float*)Q, buf, mi);
+    else out_emit_kernel<float, 64><<<nchunk, 1024, 0, s>>>(dims, (const float*)Q, buf, mi);
+  } else {
+    if (dims.d == 16) out_emit_kernel<__nv_bfloat16, 16><<<nchunk, 1024, 0, s>>>(dims, (const __nv_bfloat16*)Q, buf, mi);
+    else out_emit_kernel<__nv_bfloat16, 64><<<nchunk, 1024, 0, s>>>(dims, (const __nv_bfloat16*)Q, buf, mi);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dense_items(const Dims& dims, const Buffers& buf, cudaStream_t s) {
+  dense_items_kernel<<<148, 256, 0, s>>>(dims, buf);
+  return cudaGetLastError();
+}
+
+}  // namespace httm
