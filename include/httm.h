@@ -235,6 +235,39 @@ typedef enum {
 httm_status httm_profile_enable(httm_plan_t plan, int enable);
 httm_status httm_profile_read(httm_plan_t plan, float* ms, int32_t* launches);
 
+/*
+ * httm_select_outliers_noalloc: the global outlier selection of the filter
+ * stage, for callers that cannot allocate device memory -- code running
+ * inside a host application or inference runtime that hands it only input
+ * and output buffers and owns every allocation itself, or a latency-critical
+ * loop where a cudaMalloc could synchronise the device or fail under memory
+ * pressure.  The HTTM note has no counterpart of this entry point; it exists
+ * for those callers only.
+ *
+ * It allocates nothing: no cudaMalloc/cudaFree and no allocating library
+ * routine.  Its scratch (selection histograms, per-chunk counts, counters,
+ * about 157 KB) is a fixed array inside the library that every GPU which
+ * loads the library holds until the process exits.  Every call on a device
+ * shares that one array, and each call clears what must start at zero, so
+ * consecutive calls are independent -- but calls that overlap on the GPU
+ * (different streams, or different host threads, at the same time) race and
+ * give undefined results.  The first call on each device looks up the
+ * array's device address (a host-side set-up step, done once per device);
+ * make that first call before any stream capture.
+ *
+ * Inputs (device): dev [h, N] fp32, each query's deviation from its merged
+ * token (finite, >= 0 where eligible); eligible [h, N] u8, nonzero for
+ * queries in a merged group of >= 2 tokens.  It selects
+ * k = min(floor(outlier_pct * h * N / 100), #eligible) eligible queries with
+ * the largest deviation, ties to the lower flat index h * N + n -- the same
+ * mask httm_forward_debug exports -- and writes mask [h, N] u8 (1 = outlier)
+ * and n_out [h] int32 (outliers per head).  Limits: h <= 64 and
+ * h * N <= 33,554,432 tokens; larger sizes return HTTM_ERR_UNSUPPORTED and
+ * enqueue nothing.  Asynchronous on `stream`.
+ */
+httm_status httm_select_outliers_noalloc(const float* dev, const uint8_t* eligible, int32_t h, int32_t N,
+                                         int32_t outlier_pct, uint8_t* mask, int32_t* n_out, void* stream);
+
 const char* httm_status_str(httm_status s);
 
 #ifdef __cplusplus

@@ -26,7 +26,7 @@ EXPORTS = (
     "httm_plan", "httm_plan_destroy", "httm_get_plan_info", "httm_workspace_bytes",
     "httm_forward", "httm_forward_debug", "httm_forward_with_plan", "httm_reorder",
     "httm_get_device_status", "httm_forward_launches", "httm_profile_enable", "httm_profile_read",
-    "httm_status_str",
+    "httm_select_outliers_noalloc", "httm_status_str",
 )
 STAGES = ("match", "merge", "outlier", "attention", "unmerge", "other")
 
@@ -88,6 +88,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.httm_forward_launches.restype = ctypes.c_int32
     lib.httm_profile_enable.argtypes = [P, I]
     lib.httm_profile_read.argtypes = [P, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int32)]
+    lib.httm_select_outliers_noalloc.argtypes = [V, V, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, V, V, V]
+    lib.httm_select_outliers_noalloc.restype = ctypes.c_int
     lib.httm_status_str.argtypes = [I]
     lib.httm_status_str.restype = ctypes.c_char_p
     for name in ("httm_plan", "httm_get_plan_info", "httm_forward", "httm_forward_debug",
@@ -296,3 +298,19 @@ def workspace_view(plan: Plan, workspace, which: str):
         off = info.ws_k_tilde if which == "k" else info.ws_v_tilde
         rows = plan.cfg.h * info.kv_slots
     return workspace[off:off + rows * d * es].view(plan.dtype).view(rows, d)
+
+
+def httm_select_outliers_noalloc(dev, eligible, outlier_pct: int, mask=None, n_out=None, stream=None):
+    """Outlier selection that allocates no device memory inside the library
+    (its scratch is a fixed array in the library).  dev: [h, N] fp32 CUDA
+    tensor, eligible: [h, N] uint8.  Returns (mask [h, N] uint8, n_out [h]
+    int32).  Calls that overlap on the GPU race (they share the scratch)."""
+    h, N = dev.shape
+    if dev.dtype != torch.float32 or eligible.dtype != torch.uint8 or eligible.shape != dev.shape:
+        raise ValueError("dev must be float32 [h, N] and eligible uint8 [h, N]")
+    mask = torch.empty((h, N), dtype=torch.uint8, device=dev.device) if mask is None else mask
+    n_out = torch.empty((h,), dtype=torch.int32, device=dev.device) if n_out is None else n_out
+    _check(load_library().httm_select_outliers_noalloc(_ptr(dev), _ptr(eligible), h, N, outlier_pct, _ptr(mask),
+                                                       _ptr(n_out), _stream(stream)),
+           "httm_select_outliers_noalloc")
+    return mask, n_out
