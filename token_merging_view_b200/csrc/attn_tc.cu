@@ -1,11 +1,322 @@
-// Tensor-core (tcgen05) attention: placeholder until the kernel lands.
+// softmax(Q~ K~^T * scale) V~ on tensor cores (tcgen05 + TMEM + TMA), bf16,
+// d_head = 64.
+//
+// "HTTM: Head-wise Temporal Token Merging for Faster VGGT", overall framework
+// and training-strategy section: after merging, attention runs per head on
+// the shortened Q~/K~/V~ in bf16 with a FlashAttention-style kernel.  The
+// same kernel is the library's dense attention (HTTM_DENSE).
+//
+// One CTA per work item (a tile of <= 128 query rows of one head), 6 warps:
+//   warp 0      TMA producer: the Q tile once, then K/V tiles of 128 keys
+//               into a 3-stage shared-memory ring;
+//   warp 1      one thread issues tcgen05.mma: S_j = Q K_j^T into one of two
+//               TMEM buffers (M=128, N=128, K=64), then O += P_j V_j
+//               (M=128, N=64, K=128) into a TMEM accumulator;
+//   warps 2..5  softmax, one query row per thread (TMEM lane = row): read
+//               S_j from TMEM, running max in base 2, P_j = 2^(s*c - m) as
+//               bf16 into shared memory for the next MMA, running sum in fp32.
+// The running max is updated lazily: O and the sum are rescaled only when a
+// row's max grows by more than 8 (in log2 units), so most tiles never touch
+// O; P stays below 2^8 and every sum stays in fp32.  QK of tile j+1 overlaps
+// the softmax of tile j.  Every wait is bounded (2 s): a wait that runs out
+// sets HTTM_DEV_TIMEOUT, the CTA drains its MMAs, frees TMEM and exits.
+#include <mutex>
+
 #include "common.cuh"
 #include "launch.h"
+#include "tc_ptx.cuh"
 
 namespace httm {
-bool attention_tc_supported(const Dims&, bool) { return false; }
-cudaError_t launch_attention_tc(const Dims&, const void*, const void*, const void*, void*, int, const Buffers&,
-                                cudaStream_t) {
-  return cudaErrorNotSupported;
+namespace {
+
+using namespace tc;
+
+constexpr int kBM = 128;
+constexpr int kBN = 128;
+constexpr int kD = 64;
+constexpr int kStages = 3;
+constexpr int kThreads = 192;
+constexpr uint32_t kTile = kBN * kD * 2;   // 16 KB: 128 rows x 64 bf16
+
+struct AttnSmem {
+  uint8_t q[kTile];
+  uint8_t k[kStages][kTile];
+  uint8_t v[kStages][kTile];
+  uint8_t p[2][2 * kTile];                 // P_j: keys 0-63 then 64-127, each a K-major SW128 tile
+  uint64_t q_full;
+  uint64_t kv_full[kStages], kv_empty[kStages];
+  uint64_t s_full[2], s_free[2], p_full[2], o_done[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+constexpr size_t kSmemBytes = sizeof(AttnSmem) + 1024;
+
+// Bounded wait that ignores the abort flag (used to drain in-flight MMAs).
+__device__ bool drain_wait(uint64_t* bar, uint32_t parity) {
+  const unsigned long long t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity))
+    if (globaltimer() - t0 > kWaitTimeoutNs) return false;
+  return true;
 }
+
+__global__ void __launch_bounds__(kThreads, 1)
+attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+               const __grid_constant__ CUtensorMap tv, __nv_bfloat16* __restrict__ O, int Lk, float scale_log2,
+               Buffers buf) {
+  if (blockIdx.x >= buf.state->n_items) return;
+  if (cta_plan_failed(buf.state)) return;
+  extern __shared__ uint8_t smem_raw[];
+  AttnSmem& sm = *reinterpret_cast<AttnSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int4 it = buf.items[blockIdx.x];
+  const int hh = it.x, q_row0 = it.y, n_rows = it.z;
+  const int kv_row0 = hh * Lk;
+  const int n_kv = (Lk + kBN - 1) / kBN;
+  DevState* st = buf.state;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&sm.q_full, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sm.kv_full[s], 1);
+      mbar_init(&sm.kv_empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sm.s_full[b], 1);
+      mbar_init(&sm.s_free[b], 128);
+      mbar_init(&sm.p_full[b], 128);
+      mbar_init(&sm.o_done[b], 1);
+    }
+    mbar_init(&sm.drain, 1);
+    sm.abort = 0;
+    mbar_fence_init();
+  }
+  if (warp == 0) tmem_alloc(&sm.tmem_base, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* abort = &sm.abort;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ producer
+      tma_prefetch_desc(&tq);
+      tma_prefetch_desc(&tk);
+      tma_prefetch_desc(&tv);
+      mbar_arrive_expect_tx(&sm.q_full, kTile);
+      tma_load_2d(sm.q, &tq, &sm.q_full, 0, q_row0);
+      for (int j = 0; j < n_kv; ++j) {
+        const int s = j % kStages;
+        if (j >= kStages && !mbar_wait(&sm.kv_empty[s], ((j / kStages) - 1) & 1, abort, st)) break;
+        mbar_arrive_expect_tx(&sm.kv_full[s], 2 * kTile);
+        tma_load_2d(sm.k[s], &tk, &sm.kv_full[s], 0, kv_row0 + j * kBN);
+        tma_load_2d(sm.v[s], &tv, &sm.kv_full[s], 0, kv_row0 + j * kBN);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ MMA issue
+      constexpr uint32_t id_s = idesc_bf16(kBM, kBN, false, false);
+      constexpr uint32_t id_o = idesc_bf16(kBM, kD, false, true);
+      const uint32_t q_addr = smem_u32(sm.q);
+      bool ok = mbar_wait(&sm.q_full, 0, abort, st);
+      auto issue_qk = [&](int j) -> bool {
+        const int s = j % kStages;
+        if (!mbar_wait(&sm.kv_full[s], (j / kStages) & 1, abort, st)) return false;
+        if (j >= 2 && !mbar_wait(&sm.s_free[j & 1], ((j - 2) >> 1) & 1, abort, st)) return false;
+        tc_fence_after();
+        const uint32_t k_addr = smem_u32(sm.k[s]);
+        const uint32_t d = tmem + (uint32_t)(j & 1) * kBN;
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk)
+          umma_bf16(d, sw128_desc(q_addr + kk * 32, 1024), sw128_desc(k_addr + kk * 32, 1024), id_s, kk > 0);
+        umma_commit(&sm.s_full[j & 1]);
+        return true;
+      };
+      if (ok) ok = issue_qk(0);
+      for (int j = 0; ok && j < n_kv; ++j) {
+        if (j + 1 < n_kv && !issue_qk(j + 1)) break;
+        if (!mbar_wait(&sm.p_full[j & 1], (j >> 1) & 1, abort, st)) break;
+        tc_fence_after();
+        const int s = j % kStages;
+        const uint32_t p_addr = smem_u32(sm.p[j & 1]);
+        const uint32_t v_addr = smem_u32(sm.v[s]);
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          umma_bf16(tmem + 2 * kBN, sw128_desc(p_addr + (kk >> 2) * kTile + (kk & 3) * 32, 1024),
+                    sw128_desc(v_addr + kk * 16 * 128, 1024), id_o, (j > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(&sm.o_done[j & 1]);
+        umma_commit(&sm.kv_empty[s]);
+      }
+      // every MMA issued above completes before TMEM is released
+      umma_commit(&sm.drain);
+      drain_wait(&sm.drain, 0);
+    }
+  } else {
+    // -------------------------------------------------------------- softmax
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_kv; ++j) {
+      const int b = j & 1;
+      // waits are made warp-uniform: tcgen05.ld/st below need every lane
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[b], (j >> 1) & 1, abort, st))) { ok = false; break; }
+      tc_fence_after();
+      uint32_t sr[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        tmem_ld32(tmem + lane_off + (uint32_t)(b * kBN + c * 32), *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&sm.s_free[b]);
+      const int valid = Lk - j * kBN;
+      if (valid < kBN) {
+#pragma unroll
+        for (int i = 0; i < kBN; ++i)
+          if (i >= valid) sr[i] = __float_as_uint(-INFINITY);
+      }
+      float mt = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < kBN; ++i) mt = fmaxf(mt, __uint_as_float(sr[i]));
+      const float mts = mt * scale_log2;
+      const bool need = mts > m_used + 8.f;
+      if (__any_sync(0xffffffffu, need)) {
+        const float m_new = fmaxf(m_used, mts);
+        const float alpha = ex2(m_used - m_new);
+        if (j > 0) {
+          if (!__all_sync(0xffffffffu, mbar_wait(&sm.o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort, st))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            uint32_t o[32];
+            const uint32_t ta = tmem + lane_off + (uint32_t)(2 * kBN + c * 32);
+            tmem_ld32(ta, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(ta, o);
+          }
+          tmem_wait_st();
+        }
+        l *= alpha;
+        m_used = m_new;
+      }
+      if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(&sm.o_done[b], ((j - 2) >> 1) & 1, abort, st))) {
+        ok = false;
+        break;
+      }
+      uint8_t* prow = sm.p[b] + (row >> 3) * 1024 + (row & 7) * 128;
+      float rs = 0.f;
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float p0 = ex2(fmaf(__uint_as_float(sr[c * 8 + 2 * e]), scale_log2, -m_used));
+          const float p1 = ex2(fmaf(__uint_as_float(sr[c * 8 + 2 * e + 1]), scale_log2, -m_used));
+          rs += p0 + p1;
+          w[e] = pack_bf16(p0, p1);
+        }
+        const int cc = c & 7;
+        *reinterpret_cast<uint4*>(prow + (c >> 3) * kTile + ((cc ^ (row & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      l += rs;
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(&sm.p_full[b]);
+    }
+    if (ok && __all_sync(0xffffffffu, mbar_wait(&sm.o_done[(n_kv - 1) & 1], ((n_kv - 1) >> 1) & 1, abort, st))) {
+      tc_fence_after();
+      const float inv = 1.f / l;
+      uint32_t packed[32];
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tmem + lane_off + (uint32_t)(2 * kBN + c * 32), o);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          packed[c * 16 + i] = pack_bf16(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
+      }
+      if (row < n_rows) {
+        uint4* dst = reinterpret_cast<uint4*>(O + ((size_t)q_row0 + row) * kD);
+#pragma unroll
+        for (int v = 0; v < 8; ++v)
+          dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    if (*abort) {
+      // let TMA copies still in flight land before the shared memory goes away
+      for (int i = 0; i < 200; ++i) __nanosleep(1000);
+    }
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// [rows, 64] bf16 row-major, 128-row x 64-column boxes, 128-byte swizzle;
+// rows past the end read as zero.
+bool map_rows64(CUtensorMap* m, const void* base, uint64_t rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)kD * 2};
+  cuuint32_t box[2] = {(cuuint32_t)kD, 128};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool tma_encode_available() { return encode_fn() != nullptr; }
+
+bool attention_tc_supported(const Dims& dims, bool fp32) {
+  return !fp32 && dims.d == kD && tma_encode_available();
+}
+
+cudaError_t launch_attention_tc(const Dims& dims, const void* q, const void* k, const void* v, void* o, int Lk,
+                                const Buffers& buf, cudaStream_t s) {
+  CUtensorMap tq, tk, tv;
+  const uint64_t q_rows = dims.mode == HTTM_DENSE ? (uint64_t)dims.h * dims.N : (uint64_t)dims.q_rows_alloc;
+  const uint64_t kv_rows = (uint64_t)dims.h * Lk;
+  if (!map_rows64(&tq, q, q_rows) || !map_rows64(&tk, k, kv_rows) || !map_rows64(&tv, v, kv_rows))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+  if (e != cudaSuccess) return e;
+  const float scale_log2 = dims.scale * 1.4426950408889634f;
+  attn_tc_kernel<<<dims.max_items, kThreads, kSmemBytes, s>>>(tq, tk, tv, static_cast<__nv_bfloat16*>(o), Lk,
+                                                              scale_log2, buf);
+  return cudaGetLastError();
+}
+
 }  // namespace httm
