@@ -22,6 +22,9 @@ struct httm_plan_s {
   BlockDesc* blocks_d = nullptr;
   int4* match_items_d = nullptr;
   int n_match_items = 0;
+  int4* tc_items_d = nullptr;   // tensor-core matching: (tensor + 2 * head, block, first source, sources)
+  int n_tc_items = 0;
+  std::vector<int4> tc_items_h;
   Workspace ws;
   int launches = 0;
   std::vector<int4> items_h;
@@ -155,16 +158,23 @@ httm_status check_device(httm_plan_s* plan) {
     if (plan->dims.mode != HTTM_DENSE) {
       const size_t nb = plan->blocks_h.size() * sizeof(BlockDesc);
       const size_t ni = std::max<size_t>(1, plan->items_h.size()) * sizeof(int4);
+      const size_t nt = std::max<size_t>(1, plan->tc_items_h.size()) * sizeof(int4);
       if (cudaMalloc(&plan->blocks_d, nb) != cudaSuccess ||
           cudaMemcpy(plan->blocks_d, plan->blocks_h.data(), nb, cudaMemcpyHostToDevice) != cudaSuccess ||
           cudaMalloc(&plan->match_items_d, ni) != cudaSuccess ||
           (!plan->items_h.empty() &&
            cudaMemcpy(plan->match_items_d, plan->items_h.data(), plan->items_h.size() * sizeof(int4),
+                      cudaMemcpyHostToDevice) != cudaSuccess) ||
+          cudaMalloc(&plan->tc_items_d, nt) != cudaSuccess ||
+          (!plan->tc_items_h.empty() &&
+           cudaMemcpy(plan->tc_items_d, plan->tc_items_h.data(), plan->tc_items_h.size() * sizeof(int4),
                       cudaMemcpyHostToDevice) != cudaSuccess)) {
         if (plan->blocks_d) cudaFree(plan->blocks_d);
         if (plan->match_items_d) cudaFree(plan->match_items_d);
+        if (plan->tc_items_d) cudaFree(plan->tc_items_d);
         plan->blocks_d = nullptr;
         plan->match_items_d = nullptr;
+        plan->tc_items_d = nullptr;
         return HTTM_ERR_CUDA;
       }
     }
@@ -236,7 +246,7 @@ httm_status forward_impl(httm_plan_s* plan, const void* Q, const void* K, const 
     StageTimer t(plan, s, HTTM_STAGE_MATCH, 1);
     cudaError_t e = cudaErrorNotSupported;
     if (match_tc_supported(dims, fp32))
-      e = launch_match_tc(dims, plan->blocks_d, plan->match_items_d, plan->n_match_items, Q, K, buf, s);
+      e = launch_match_tc(dims, plan->blocks_d, plan->tc_items_d, plan->n_tc_items, Q, K, buf, s);
     else
       e = launch_match_simt(dims, fp32, plan->blocks_d, plan->match_items_d, plan->n_match_items, Q, K, buf, s);
     ++launches;
@@ -406,6 +416,30 @@ httm_status httm_plan(const httm_cfg* cfg, httm_plan_t* out) {
     });
     p->n_match_items = (int)items.size();
     p->items_h = std::move(items);
+    // tensor-core matching: one CTA per (tensor, head, block), a block split in
+    // runs of whole 128-source tiles when that gives too few CTAs; costliest first
+    std::vector<int4> tci;
+    const int parts_want = std::max(1, (4 * 148 + 2 * d.nblk * c.h - 1) / (2 * d.nblk * c.h));
+    for (int hh = 0; hh < c.h; ++hh)
+      for (int t = 0; t < 2; ++t)
+        for (int bi = 0; bi < d.nblk; ++bi) {
+          const BlockDesc& b = B[bi];
+          const int ns = b.n_b - (t == 0 ? b.q_ndst : b.k_ndst);
+          const int tiles = (ns + 127) / 128;
+          const int parts = std::max(1, std::min(parts_want, tiles));
+          const int per = (tiles + parts - 1) / parts;
+          for (int t0 = 0; t0 < tiles; t0 += per) {
+            const int s0 = t0 * 128, n = std::min(per * 128, ns - s0);
+            tci.push_back(make_int4(t + 2 * hh, bi, s0, n));
+          }
+        }
+    std::stable_sort(tci.begin(), tci.end(), [&](const int4& a, const int4& b) {
+      const long long ca = (long long)((a.x & 1) == 0 ? B[a.y].q_ndst : B[a.y].k_ndst) * a.w;
+      const long long cb = (long long)((b.x & 1) == 0 ? B[b.y].q_ndst : B[b.y].k_ndst) * b.w;
+      return ca > cb;
+    });
+    p->n_tc_items = (int)tci.size();
+    p->tc_items_h = std::move(tci);
   }
   p->ws = layout(d, p->fp32);
   *out = p;
@@ -421,6 +455,7 @@ void httm_plan_destroy(httm_plan_t plan) {
   for (cudaEvent_t e : plan->pool) cudaEventDestroy(e);
   if (plan->blocks_d) cudaFree(plan->blocks_d);
   if (plan->match_items_d) cudaFree(plan->match_items_d);
+  if (plan->tc_items_d) cudaFree(plan->tc_items_d);
   delete plan;
 }
 

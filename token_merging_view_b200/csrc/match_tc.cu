@@ -1,11 +1,303 @@
-// Tensor-core (tcgen05) matching: placeholder until the kernel lands.
+// Bipartite cosine matching on tensor cores (tcgen05 + TMEM), bf16, d = 64.
+//
+// "HTTM: Head-wise Temporal Token Merging for Faster VGGT", key design 1:
+// per head, Sim = RowNorm(S) . RowNorm(D)^T and every source keeps only its
+// most similar destination; key design 2: only inside a block.  Here the
+// block's raw source/destination rows feed the MMA (bf16 products are exact,
+// sums are fp32), and the normalisation moves to the epilogue:
+// argmax_t dot(s, t) / ||t||, score = that / ||s||, so the n_src x n_dst
+// similarity matrix never leaves the SM.
+//
+// One CTA per (tensor, head, block, run of 128-source tiles), 9 warps:
+//   warps 0..7  gather rows with cp.async into the 128-byte-swizzled operand
+//               layout (all destinations of the block once, then source tiles
+//               double-buffered), compute norms, and run the epilogue: warp w
+//               reads TMEM lanes 32*(w%4).. (one source row per thread) and the
+//               column half w/4 of each chunk; running (max, first index);
+//   warp 8      allocates TMEM and one thread issues tcgen05.mma: for each
+//               source tile, destination chunks of <= 256 columns into two
+//               TMEM buffers of 256 fp32 columns.
+// Ties keep the lowest destination (strict '>' in ascending column order;
+// the lower column half wins equal values).  Every wait is bounded.
 #include "common.cuh"
 #include "launch.h"
+#include "tc_ptx.cuh"
 
 namespace httm {
-bool match_tc_supported(const Dims&, bool) { return false; }
-cudaError_t launch_match_tc(const Dims&, const BlockDesc*, const int4*, int, const void*, const void*,
-                            const Buffers&, cudaStream_t) {
-  return cudaErrorNotSupported;
+namespace {
+
+using namespace tc;
+
+constexpr int kEpiThreads = 256;
+constexpr int kThreads = kEpiThreads + 32;
+constexpr int kMaxDst = 1024;          // destination rows a block may have on this path
+constexpr int kChunkCols = 256;
+constexpr uint32_t kRowsTile = 128;
+constexpr uint32_t kTileBytes = kRowsTile * 128;
+
+struct MatchSmem {
+  uint8_t dst[kMaxDst * 128];          // K-major SW128, 128 KB
+  uint8_t src[2][kTileBytes];
+  float inv_d[kMaxDst];
+  float best_v[2][128];
+  int best_i[2][128];
+  uint64_t src_ready[2], full[2], empty[2], drain;
+  uint32_t tmem_base;
+  int abort;
+};
+constexpr size_t kSmemBytes = sizeof(MatchSmem) + 1024;
+
+__device__ __forceinline__ uint32_t swz(uint32_t row, uint32_t chunk) {
+  return (row >> 3) * 1024u + (row & 7u) * 128u + ((chunk ^ (row & 7u)) << 4);
 }
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
+  const uint32_t n = valid ? 16u : 0u;
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(n) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory"); }
+
+__device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
+  const unsigned long long t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity))
+    if (globaltimer() - t0 > kWaitTimeoutNs) return false;
+  return true;
+}
+
+// item: tensor (0 = Q, 1 = K) + 2 * head, block, first source ordinal, sources
+__global__ void __launch_bounds__(kThreads, 1)
+match_tc_kernel(Dims dims, const BlockDesc* __restrict__ blocks, const int4* __restrict__ items,
+                const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K, Buffers buf) {
+  extern __shared__ uint8_t smem_raw[];
+  MatchSmem& sm = *reinterpret_cast<MatchSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int4 it = items[blockIdx.x];
+  const int hh = it.x >> 1;
+  const bool is_q = (it.x & 1) == 0;
+  const BlockDesc b = blocks[it.y];
+  const int stride = is_q ? dims.q_stride : dims.kv_stride;
+  const int ndst = is_q ? b.q_ndst : b.k_ndst;
+  const int ndst_pad = (ndst + 63) & ~63;
+  const int nchunk = (ndst_pad + kChunkCols - 1) / kChunkCols;
+  const int src0 = it.z, nsrc = it.w;
+  const int ntile = (nsrc + kRowsTile - 1) / kRowsTile;
+  const __nv_bfloat16* Xh = (is_q ? Q : K) + (size_t)hh * dims.N * 64;
+  const size_t out_base = (size_t)hh * (is_q ? dims.q_src : dims.k_src) + (is_q ? b.q_src_off : b.k_src_off);
+  int32_t* best_out = (is_q ? buf.q_best : buf.k_best) + out_base;
+  float* score_out = (is_q ? buf.q_score : buf.k_score) + out_base;
+  DevState* st = buf.state;
+
+  if (tid == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.src_ready[i], kEpiThreads);
+      mbar_init(&sm.full[i], 1);
+      mbar_init(&sm.empty[i], kEpiThreads);
+    }
+    mbar_init(&sm.drain, 1);
+    sm.abort = 0;
+    mbar_fence_init();
+  }
+  if (warp == 8) tmem_alloc(&sm.tmem_base, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* abort = &sm.abort;
+
+  if (warp == 8) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ MMA issue
+      uint32_t gc = 0;
+      bool ok = true;
+      const uint32_t dst_addr = smem_u32(sm.dst);
+      for (int t = 0; ok && t < ntile; ++t) {
+        if (!mbar_wait(&sm.src_ready[t & 1], (t >> 1) & 1, abort, st)) break;
+        tc_fence_after();
+        const uint32_t src_addr = smem_u32(sm.src[t & 1]);
+        for (int c = 0; c < nchunk; ++c, ++gc) {
+          const uint32_t bb = gc & 1;
+          if (gc >= 2 && !mbar_wait(&sm.empty[bb], ((gc - 2) >> 1) & 1, abort, st)) { ok = false; break; }
+          tc_fence_after();
+          const int width = min(kChunkCols, ndst_pad - c * kChunkCols);
+          const uint32_t idesc = idesc_bf16(128, width, false, false);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16(tmem + bb * kChunkCols, sw128_desc(src_addr + kk * 32, 1024),
+                      sw128_desc(dst_addr + c * kChunkCols * 128 + kk * 32, 1024), idesc, kk > 0);
+          umma_commit(&sm.full[bb]);
+        }
+      }
+      umma_commit(&sm.drain);
+      drain_wait(&sm.drain, 0);
+    }
+  } else {
+    // ------------------------------------------------------ gather + epilogue
+    const uint32_t dst_addr = smem_u32(sm.dst);
+    // destinations (rows padded with zeros to a multiple of 64)
+    for (int e = tid; e < ndst_pad * 8; e += kEpiThreads) {
+      const int r = e >> 3, ch = e & 7;
+      const bool valid = r < ndst;
+      const int tok = valid ? block_token(b, r * stride, dims.P) : b.base;
+      cp_async16(dst_addr + swz(r, ch), Xh + (size_t)tok * 64 + ch * 8, valid);
+    }
+    auto load_tile = [&](int t) {
+      const uint32_t base = smem_u32(sm.src[t & 1]);
+      for (int e = tid; e < (int)kRowsTile * 8; e += kEpiThreads) {
+        const int r = e >> 3, ch = e & 7;
+        const int k = src0 + t * kRowsTile + r;
+        const bool valid = t * (int)kRowsTile + r < nsrc;
+        const int tok = valid ? block_token(b, src_index(k, stride), dims.P) : b.base;
+        cp_async16(base + swz(r, ch), Xh + (size_t)tok * 64 + ch * 8, valid);
+      }
+    };
+    load_tile(0);
+    cp_async_commit();
+    const int quarter = warp & 3, half = warp >> 2;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    // Abort handling: a failed wait clears `ok` (warp-uniform) and sets the
+    // CTA's abort flag; the warp then skips its work but still reaches every
+    // named barrier, so no warp waits on one that another warp has left.
+    uint32_t gc = 0;
+    bool ok = true;
+    for (int t = 0; t < ntile; ++t) {
+      if (t + 1 < ntile) {
+        load_tile(t + 1);
+        cp_async_commit();
+        cp_async_wait<1>();
+      } else {
+        cp_async_wait<0>();
+      }
+      fence_async_smem();
+      epi_sync();
+      if (t == 0) {
+        // destination inverse norms (fp32, fixed order)
+        for (int r = tid; r < ndst_pad; r += kEpiThreads) {
+          float ss = 0.f;
+          for (int ch = 0; ch < 8; ++ch) {
+            const uint4 w = *reinterpret_cast<const uint4*>(sm.dst + swz(r, ch));
+            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const float lo = __uint_as_float(ws[q] << 16), hi = __uint_as_float(ws[q] & 0xffff0000u);
+              ss = fmaf(lo, lo, ss);
+              ss = fmaf(hi, hi, ss);
+            }
+          }
+          sm.inv_d[r] = ss > 0.f ? 1.f / sqrtf(ss) : 0.f;
+        }
+        epi_sync();
+      }
+      mbar_arrive(&sm.src_ready[t & 1]);
+      // this row's inverse norm
+      float inv_s;
+      {
+        float ss = 0.f;
+        for (int ch = 0; ch < 8; ++ch) {
+          const uint4 w = *reinterpret_cast<const uint4*>(sm.src[t & 1] + swz(row, ch));
+          const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float lo = __uint_as_float(ws[q] << 16), hi = __uint_as_float(ws[q] & 0xffff0000u);
+            ss = fmaf(lo, lo, ss);
+            ss = fmaf(hi, hi, ss);
+          }
+        }
+        inv_s = ss > 0.f ? 1.f / sqrtf(ss) : 0.f;
+      }
+      float best = -INFINITY;
+      int bi = 0;
+      for (int c = 0; c < nchunk; ++c, ++gc) {
+        const uint32_t bb = gc & 1;
+        if (ok && !__all_sync(0xffffffffu, mbar_wait(&sm.full[bb], (gc >> 1) & 1, abort, st))) {
+          ok = false;
+          *abort = 1;
+        }
+        if (!ok) continue;
+        tc_fence_after();
+        const int width = min(kChunkCols, ndst_pad - c * kChunkCols);
+        const int hw = width >> 1;                       // multiple of 32
+        const int col0 = c * kChunkCols + half * hw;
+        for (int g = 0; g < hw; g += 32) {
+          uint32_t r[32];
+          tmem_ld32(tmem + lane_off + bb * kChunkCols + half * hw + g, r);
+          tmem_wait_ld();
+          const int cb = col0 + g;
+          const float4* invp = reinterpret_cast<const float4*>(sm.inv_d + cb);
+          if (cb + 32 <= ndst) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const float4 iv = invp[q];
+              const float v0 = __uint_as_float(r[4 * q]) * iv.x, v1 = __uint_as_float(r[4 * q + 1]) * iv.y;
+              const float v2 = __uint_as_float(r[4 * q + 2]) * iv.z, v3 = __uint_as_float(r[4 * q + 3]) * iv.w;
+              if (v0 > best) { best = v0; bi = cb + 4 * q; }
+              if (v1 > best) { best = v1; bi = cb + 4 * q + 1; }
+              if (v2 > best) { best = v2; bi = cb + 4 * q + 2; }
+              if (v3 > best) { best = v3; bi = cb + 4 * q + 3; }
+            }
+          } else {
+#pragma unroll
+            for (int q = 0; q < 32; ++q) {
+              if (cb + q < ndst) {
+                const float v = __uint_as_float(r[q]) * sm.inv_d[cb + q];
+                if (v > best) { best = v; bi = cb + q; }
+              }
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&sm.empty[bb]);
+      }
+      sm.best_v[half][row] = best;
+      sm.best_i[half][row] = bi;
+      epi_sync();
+      if (half == 0 && ok) {
+        const int k = t * kRowsTile + row;
+        if (k < nsrc) {
+          // the two column halves of one row: larger value, lower index on ties
+          float v = sm.best_v[0][row];
+          int i = sm.best_i[0][row];
+          const float v1 = sm.best_v[1][row];
+          const int i1 = sm.best_i[1][row];
+          if (v1 > v || (v1 == v && i1 < i)) {
+            v = v1;
+            i = i1;
+          }
+          best_out[src0 + k] = i;
+          score_out[src0 + k] = v * inv_s;
+        }
+      }
+      epi_sync();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+bool tma_encode_available();
+
+bool match_tc_supported(const Dims& dims, bool fp32) {
+  return !fp32 && dims.d == 64 && dims.mode != HTTM_HEAD_UNIFORM && dims.max_ndst <= kMaxDst;
+}
+
+cudaError_t launch_match_tc(const Dims& dims, const BlockDesc* blocks, const int4* items, int n_items,
+                            const void* Q, const void* K, const Buffers& buf, cudaStream_t s) {
+  if (n_items == 0) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(match_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+  if (e != cudaSuccess) return e;
+  match_tc_kernel<<<n_items, kThreads, kSmemBytes, s>>>(
+      dims, blocks, items, static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K), buf);
+  return cudaGetLastError();
+}
+
 }  // namespace httm
