@@ -6,20 +6,34 @@
 // the shortened Q~/K~/V~ in bf16 with a FlashAttention-style kernel.  The
 // same kernel is the library's dense attention (HTTM_DENSE).
 //
-// One CTA per work item (a tile of <= 128 query rows of one head), 6 warps:
-//   warp 0      TMA producer: the Q tile once, then K/V tiles of 128 keys
-//               into a 3-stage shared-memory ring;
-//   warp 1      one thread issues tcgen05.mma: S_j = Q K_j^T into one of two
-//               TMEM buffers (M=128, N=128, K=64), then O += P_j V_j
-//               (M=128, N=64, K=128) into a TMEM accumulator;
-//   warps 2..5  softmax, one query row per thread (TMEM lane = row): read
-//               S_j from TMEM, running max in base 2, P_j = 2^(s*c - m) as
-//               bf16 into shared memory for the next MMA, running sum in fp32.
-// The running max is updated lazily: O and the sum are rescaled only when a
-// row's max grows by more than 8 (in log2 units), so most tiles never touch
-// O; P stays below 2^8 and every sum stays in fp32.  QK of tile j+1 overlaps
-// the softmax of tile j.  Every wait is bounded (2 s): a wait that runs out
-// sets HTTM_DEV_TIMEOUT, the CTA drains its MMAs, frees TMEM and exits.
+// One CTA per work item: up to 256 query rows of one head, as two 128-row
+// tiles t = 0, 1.  12 warps = 3 warpgroups:
+//   warp 0      TMA producer: both Q tiles once, then K/V tiles of 128 keys
+//               into a 4-stage shared-memory ring;
+//   warp 1      one thread issues tcgen05.mma:
+//                 S_t = Q_t K_j^T   (M=128, N=128, K=64; A, B in shared memory)
+//                 O_t += P_t V_j    (M=128, N=64, K=128; A = P_t in TMEM)
+//               in the order  PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1);
+//   warps 2, 3  idle;
+//   warps 4..7  softmax of tile 0, warps 8..11 softmax of tile 1: one query
+//               row per thread (TMEM lane = row).
+// Registers: launched at 168 per thread (384 x 168 = 64,512); warpgroup 0
+// gives part of its share back (setmaxnreg to 88) and the softmax warpgroups
+// take it (208): 128 x 88 + 256 x 208 = 64,512.
+// TMEM (512 columns): per tile t, S_t [t*256, +128), P_t [t*256+128, +64)
+// (bf16 pairs), O_t [t*256+192, +64).  Tensor-core operations complete in
+// issue order, so when S_t(j+1) is ready, PV_t(j) -- the last reader of P_t
+// and the last writer of O_t -- is done: the softmax may overwrite P_t and
+// rescale O_t without a further wait.  Two warpgroups keep two softmax warps
+// per SM sub-partition busy on the exp unit while the tensor core alternates
+// between the tiles.
+//
+// Softmax: base-2 running max, updated lazily -- O_t and the row sum are
+// rescaled only when the row max grows by more than 8 (log2 units), so P stays
+// below 2^8 and most tiles never touch O_t; max and sum use split
+// accumulators for instruction-level parallelism.  Every wait is bounded
+// (2 s): a wait that runs out sets HTTM_DEV_TIMEOUT, the CTA drains its MMAs,
+// frees TMEM and exits.
 #include <mutex>
 
 #include "common.cuh"
@@ -34,23 +48,24 @@ using namespace tc;
 constexpr int kBM = 128;
 constexpr int kBN = 128;
 constexpr int kD = 64;
-constexpr int kStages = 3;
-constexpr int kThreads = 192;
+constexpr int kStages = 4;
+constexpr int kThreads = 384;
 constexpr uint32_t kTile = kBN * kD * 2;   // 16 KB: 128 rows x 64 bf16
+constexpr uint32_t kColS = 0, kColP = 128, kColO = 192, kColTile = 256;
 
 struct AttnSmem {
-  uint8_t q[kTile];
+  uint8_t q[2][kTile];
   uint8_t k[kStages][kTile];
   uint8_t v[kStages][kTile];
-  uint8_t p[2][2 * kTile];                 // P_j: keys 0-63 then 64-127, each a K-major SW128 tile
   uint64_t q_full;
   uint64_t kv_full[kStages], kv_empty[kStages];
-  uint64_t s_full[2], s_free[2], p_full[2], o_done[2];
+  uint64_t s_full[2], p_full[2], o_done[2];
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
 };
 constexpr size_t kSmemBytes = sizeof(AttnSmem) + 1024;
+static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 
 // Bounded wait that ignores the abort flag (used to drain in-flight MMAs).
 __device__ bool drain_wait(uint64_t* bar, uint32_t parity) {
@@ -81,11 +96,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
       mbar_init(&sm.kv_full[s], 1);
       mbar_init(&sm.kv_empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&sm.s_full[b], 1);
-      mbar_init(&sm.s_free[b], 128);
-      mbar_init(&sm.p_full[b], 128);
-      mbar_init(&sm.o_done[b], 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&sm.s_full[t], 1);
+      mbar_init(&sm.p_full[t], 128);
+      mbar_init(&sm.o_done[t], 1);
     }
     mbar_init(&sm.drain, 1);
     sm.abort = 0;
@@ -97,15 +111,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
   volatile int* abort = &sm.abort;
-
-  if (warp == 0) {
-    if (lane == 0) {
+  if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 88;" ::: "memory");
+    if (warp == 0 && lane == 0) {
       // ------------------------------------------------------------ producer
       tma_prefetch_desc(&tq);
       tma_prefetch_desc(&tk);
       tma_prefetch_desc(&tv);
-      mbar_arrive_expect_tx(&sm.q_full, kTile);
-      tma_load_2d(sm.q, &tq, &sm.q_full, 0, q_row0);
+      mbar_arrive_expect_tx(&sm.q_full, 2 * kTile);
+      tma_load_2d(sm.q[0], &tq, &sm.q_full, 0, q_row0);
+      tma_load_2d(sm.q[1], &tq, &sm.q_full, 0, q_row0 + kBM);
       for (int j = 0; j < n_kv; ++j) {
         const int s = j % kStages;
         if (j >= kStages && !mbar_wait(&sm.kv_empty[s], ((j / kStages) - 1) & 1, abort, st)) break;
@@ -113,139 +128,139 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         tma_load_2d(sm.k[s], &tk, &sm.kv_full[s], 0, kv_row0 + j * kBN);
         tma_load_2d(sm.v[s], &tv, &sm.kv_full[s], 0, kv_row0 + j * kBN);
       }
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
+    } else if (warp == 1 && lane == 0) {
       // ------------------------------------------------------------ MMA issue
       constexpr uint32_t id_s = idesc_bf16(kBM, kBN, false, false);
       constexpr uint32_t id_o = idesc_bf16(kBM, kD, false, true);
-      const uint32_t q_addr = smem_u32(sm.q);
-      bool ok = mbar_wait(&sm.q_full, 0, abort, st);
-      auto issue_qk = [&](int j) -> bool {
-        const int s = j % kStages;
-        if (!mbar_wait(&sm.kv_full[s], (j / kStages) & 1, abort, st)) return false;
-        if (j >= 2 && !mbar_wait(&sm.s_free[j & 1], ((j - 2) >> 1) & 1, abort, st)) return false;
-        tc_fence_after();
-        const uint32_t k_addr = smem_u32(sm.k[s]);
-        const uint32_t d = tmem + (uint32_t)(j & 1) * kBN;
+      auto issue_qk = [&](int t, int j) {
+        const uint32_t q_addr = smem_u32(sm.q[t]);
+        const uint32_t k_addr = smem_u32(sm.k[j % kStages]);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk)
-          umma_bf16(d, sw128_desc(q_addr + kk * 32, 1024), sw128_desc(k_addr + kk * 32, 1024), id_s, kk > 0);
-        umma_commit(&sm.s_full[j & 1]);
-        return true;
+          umma_bf16(tmem + t * kColTile + kColS, sw128_desc(q_addr + kk * 32, 1024),
+                    sw128_desc(k_addr + kk * 32, 1024), id_s, kk > 0);
+        umma_commit(&sm.s_full[t]);
       };
-      if (ok) ok = issue_qk(0);
-      for (int j = 0; ok && j < n_kv; ++j) {
-        if (j + 1 < n_kv && !issue_qk(j + 1)) break;
-        if (!mbar_wait(&sm.p_full[j & 1], (j >> 1) & 1, abort, st)) break;
-        tc_fence_after();
-        const int s = j % kStages;
-        const uint32_t p_addr = smem_u32(sm.p[j & 1]);
-        const uint32_t v_addr = smem_u32(sm.v[s]);
+      auto issue_pv = [&](int t, int j) {
+        const uint32_t v_addr = smem_u32(sm.v[j % kStages]);
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk)
-          umma_bf16(tmem + 2 * kBN, sw128_desc(p_addr + (kk >> 2) * kTile + (kk & 3) * 32, 1024),
-                    sw128_desc(v_addr + kk * 16 * 128, 1024), id_o, (j > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(&sm.o_done[j & 1]);
-        umma_commit(&sm.kv_empty[s]);
+          umma_bf16_ts(tmem + t * kColTile + kColO, tmem + t * kColTile + kColP + kk * 8,
+                       sw128_desc(v_addr + kk * 16 * 128, 1024), id_o, (j > 0 || kk > 0) ? 1u : 0u);
+      };
+      bool ok = mbar_wait(&sm.q_full, 0, abort, st) && mbar_wait(&sm.kv_full[0], 0, abort, st);
+      if (ok) {
+        tc_fence_after();
+        issue_qk(0, 0);
+        issue_qk(1, 0);
+      }
+      for (int j = 0; ok && j < n_kv; ++j) {
+        const bool more = j + 1 < n_kv;
+        if (more && !mbar_wait(&sm.kv_full[(j + 1) % kStages], ((j + 1) / kStages) & 1, abort, st)) break;
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          if (!mbar_wait(&sm.p_full[t], j & 1, abort, st)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv(t, j);
+          if (t == 1) umma_commit(&sm.kv_empty[j % kStages]);
+          if (more) issue_qk(t, j + 1);
+          else umma_commit(&sm.o_done[t]);
+        }
       }
       // every MMA issued above completes before TMEM is released
       umma_commit(&sm.drain);
       drain_wait(&sm.drain, 0);
     }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 208;" ::: "memory");
     // -------------------------------------------------------------- softmax
+    const int t = (warp - 4) >> 2;                      // query tile of this warpgroup
     const int quarter = warp & 3;
-    const int row = quarter * 32 + lane;
+    const int row = quarter * 32 + lane;                // row inside the tile = TMEM lane
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const uint32_t ts = tmem + lane_off + t * kColTile;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n_kv; ++j) {
-      const int b = j & 1;
       // waits are made warp-uniform: tcgen05.ld/st below need every lane
-      if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[b], (j >> 1) & 1, abort, st))) { ok = false; break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[t], j & 1, abort, st))) { ok = false; break; }
       tc_fence_after();
       uint32_t sr[128];
 #pragma unroll
       for (int c = 0; c < 4; ++c)
-        tmem_ld32(tmem + lane_off + (uint32_t)(b * kBN + c * 32), *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+        tmem_ld32(ts + kColS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
       tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(&sm.s_free[b]);
       const int valid = Lk - j * kBN;
       if (valid < kBN) {
 #pragma unroll
         for (int i = 0; i < kBN; ++i)
           if (i >= valid) sr[i] = __float_as_uint(-INFINITY);
       }
-      float mt = -INFINITY;
+      float mx[8];
 #pragma unroll
-      for (int i = 0; i < kBN; ++i) mt = fmaxf(mt, __uint_as_float(sr[i]));
+      for (int a = 0; a < 8; ++a) mx[a] = __uint_as_float(sr[a]);
+#pragma unroll
+      for (int i = 8; i < kBN; ++i) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(sr[i]));
+      const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
       const float mts = mt * scale_log2;
       const bool need = mts > m_used + 8.f;
       if (__any_sync(0xffffffffu, need)) {
         const float m_new = fmaxf(m_used, mts);
         const float alpha = ex2(m_used - m_new);
         if (j > 0) {
-          if (!__all_sync(0xffffffffu, mbar_wait(&sm.o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort, st))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
+          // PV_t(j-1) completed before S_t(j) was signalled
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
             uint32_t o[32];
-            const uint32_t ta = tmem + lane_off + (uint32_t)(2 * kBN + c * 32);
-            tmem_ld32(ta, o);
+            tmem_ld32(ts + kColO + c * 32, o);
             tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st32(ta, o);
+            tmem_st32(ts + kColO + c * 32, o);
           }
-          tmem_wait_st();
         }
         l *= alpha;
         m_used = m_new;
       }
-      if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(&sm.o_done[b], ((j - 2) >> 1) & 1, abort, st))) {
-        ok = false;
-        break;
-      }
-      uint8_t* prow = sm.p[b] + (row >> 3) * 1024 + (row & 7) * 128;
-      float rs = 0.f;
+      const float neg_m = -m_used;
+      float rs[8];
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        uint32_t w[4];
+      for (int a = 0; a < 8; ++a) rs[a] = 0.f;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float p0 = ex2(fmaf(__uint_as_float(sr[c * 8 + 2 * e]), scale_log2, -m_used));
-          const float p1 = ex2(fmaf(__uint_as_float(sr[c * 8 + 2 * e + 1]), scale_log2, -m_used));
-          rs += p0 + p1;
-          w[e] = pack_bf16(p0, p1);
+      for (int c = 0; c < 2; ++c) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float p0 = ex2(fmaf(__uint_as_float(sr[c * 64 + 2 * i]), scale_log2, neg_m));
+          const float p1 = ex2(fmaf(__uint_as_float(sr[c * 64 + 2 * i + 1]), scale_log2, neg_m));
+          rs[(2 * i) & 7] += p0;
+          rs[(2 * i + 1) & 7] += p1;
+          pk[i] = pack_bf16(p0, p1);
         }
-        const int cc = c & 7;
-        *reinterpret_cast<uint4*>(prow + (c >> 3) * kTile + ((cc ^ (row & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+        tmem_st32(ts + kColP + c * 32, pk);
       }
-      l += rs;
-      fence_async_smem();
+      l += ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
+      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&sm.p_full[b]);
+      mbar_arrive(&sm.p_full[t]);
     }
-    if (ok && __all_sync(0xffffffffu, mbar_wait(&sm.o_done[(n_kv - 1) & 1], ((n_kv - 1) >> 1) & 1, abort, st))) {
+    if (ok && __all_sync(0xffffffffu, mbar_wait(&sm.o_done[t], 0, abort, st))) {
       tc_fence_after();
       const float inv = 1.f / l;
       uint32_t packed[32];
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t o[32];
-        tmem_ld32(tmem + lane_off + (uint32_t)(2 * kBN + c * 32), o);
+        tmem_ld32(ts + kColO + c * 32, o);
         tmem_wait_ld();
 #pragma unroll
         for (int i = 0; i < 16; ++i)
           packed[c * 16 + i] = pack_bf16(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
       }
-      if (row < n_rows) {
-        uint4* dst = reinterpret_cast<uint4*>(O + ((size_t)q_row0 + row) * kD);
+      const int r = t * kBM + row;
+      if (r < n_rows) {
+        uint4* dst = reinterpret_cast<uint4*>(O + ((size_t)q_row0 + r) * kD);
 #pragma unroll
         for (int v = 0; v < 8; ++v)
           dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);

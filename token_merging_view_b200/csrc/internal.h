@@ -41,7 +41,7 @@ struct Dims {
 
 constexpr int kChunk = 4096;       // keys per chunk of the outlier compaction
 constexpr int kHistBins = 2048;    // radix digit of the outlier select (11 bits)
-constexpr int kAttnRows = 128;     // query rows per attention work item
+constexpr int kAttnRows = 256;     // query rows per attention work item (two 128-row tiles)
 
 // Device-side state at the head of the workspace.
 struct DevState {
