@@ -19,7 +19,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 def _declared():
     src = open(os.path.join(ROOT, "include", "httm.h")).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(httm_[a-z_]+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b(httm_[a-z_0-9]+)\s*\(", src)))
 
 
 def test_library_exports_every_declared_symbol():

@@ -114,6 +114,30 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* tmp, u
   return r;
 }
 
+// One full warp: the bin holding the k-th largest element (k >= 1) of a
+// histogram hist[0, nb), scanned from the top bin down, and k minus the
+// number of elements in higher bins.  Every lane gets the result.
+__device__ __forceinline__ void warp_select_bin(const uint32_t* hist, int nb, uint32_t k, int* bin, uint32_t* krem) {
+  const int lane = threadIdx.x & 31;
+  uint32_t above = 0;
+  for (int top = nb - 1; top >= 0; top -= 32) {
+    const int bb = top - lane;
+    const uint32_t c = bb >= 0 ? hist[bb] : 0u;
+    const uint32_t inc = warp_incl_scan(c);
+    const uint32_t tot = __shfl_sync(0xffffffffu, inc, 31);
+    if (above + tot >= k) {
+      const unsigned ballot = __ballot_sync(0xffffffffu, above + inc >= k);
+      const int l = __ffs(ballot) - 1;
+      *bin = top - l;
+      *krem = k - (above + __shfl_sync(0xffffffffu, inc, l) - __shfl_sync(0xffffffffu, c, l));
+      return;
+    }
+    above += tot;
+  }
+  *bin = 0;
+  *krem = 0;
+}
+
 // Bitonic sort (ascending) of n = 2^k 64-bit keys in shared memory by the
 // whole thread block.
 __device__ __forceinline__ void block_bitonic_sort(unsigned long long* a, int n) {

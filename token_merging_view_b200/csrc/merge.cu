@@ -22,7 +22,7 @@
 namespace httm {
 namespace {
 
-constexpr int kMergeThreads = 512;
+constexpr int kMergeThreads = 256;
 
 // A [D]-row spread over one warp: lane l owns elements [l*E, l*E + E).
 template <class T, int D>
@@ -54,6 +54,85 @@ struct WarpRow<__nv_bfloat16, 64> {
   }
 };
 
+// A row as 16-byte chunks spread over a warp: CPR chunks per row, RPI rows
+// per warp-wide access, EPC elements per chunk.
+template <class T, int D>
+struct Chunk {
+  static constexpr int EPC = 16 / (int)sizeof(T);
+  static constexpr int CPR = D / EPC;
+  static constexpr int RPI = 32 / CPR;
+  static_assert(CPR >= 1 && CPR <= 32 && 32 % CPR == 0, "row must split into 16-byte chunks over a warp");
+  __device__ static uint4 load(const T* row, int ch) { return __ldg(reinterpret_cast<const uint4*>(row) + ch); }
+  __device__ static void unpack(const uint4& w, float (&v)[EPC]) {
+    if constexpr (sizeof(T) == 2) {
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        v[2 * q] = __uint_as_float(ws[q] << 16);
+        v[2 * q + 1] = __uint_as_float(ws[q] & 0xffff0000u);
+      }
+    } else {
+      v[0] = __uint_as_float(w.x); v[1] = __uint_as_float(w.y);
+      v[2] = __uint_as_float(w.z); v[3] = __uint_as_float(w.w);
+    }
+  }
+  __device__ static void add(float (&acc)[EPC], const uint4& w) {
+    float v[EPC];
+    unpack(w, v);
+#pragma unroll
+    for (int e = 0; e < EPC; ++e) acc[e] += v[e];
+  }
+  __device__ static float sq_dist(const uint4& w, const float (&mean)[EPC]) {
+    float v[EPC];
+    unpack(w, v);
+    float ss = 0.f;
+#pragma unroll
+    for (int e = 0; e < EPC; ++e) {
+      const float d = v[e] - mean[e];
+      ss = fmaf(d, d, ss);
+    }
+    return ss;
+  }
+  // Sum over the RPI lanes holding the same chunk of different rows; every
+  // lane gets the same bits (the butterfly is symmetric).
+  __device__ static float across_rows(float v) {
+#pragma unroll
+    for (int o = CPR; o < 32; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+  }
+  // Sum over the CPR lanes holding one row.
+  __device__ static float within_row(float v) {
+#pragma unroll
+    for (int o = 1; o < CPR; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+  }
+  __device__ static void store(T* row, int ch, const float (&v)[EPC]) {
+    uint4 w;
+    if constexpr (sizeof(T) == 2) {
+      uint32_t ws[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const __nv_bfloat162 p = __floats2bfloat162_rn(v[2 * q], v[2 * q + 1]);
+        ws[q] = *reinterpret_cast<const uint32_t*>(&p);
+      }
+      w = make_uint4(ws[0], ws[1], ws[2], ws[3]);
+    } else {
+      w = make_uint4(__float_as_uint(v[0]), __float_as_uint(v[1]), __float_as_uint(v[2]), __float_as_uint(v[3]));
+    }
+    reinterpret_cast<uint4*>(row)[ch] = w;
+  }
+  __device__ static void store_raw(T* row, int ch, const uint4& w) { reinterpret_cast<uint4*>(row)[ch] = w; }
+  __device__ static void store_f32(float* row, int ch, const float (&v)[EPC]) {
+#pragma unroll
+    for (int e = 0; e < EPC; ++e) row[ch * EPC + e] = v[e];
+  }
+  __device__ static void store_raw_f32(float* row, int ch, const uint4& w) {
+    float v[EPC];
+    unpack(w, v);
+    store_f32(row, ch, v);
+  }
+};
+
 template <int E>
 __device__ __forceinline__ void store_f32(float* row, int lane, int D, const float (&v)[E]) {
 #pragma unroll
@@ -79,17 +158,23 @@ __device__ void block_scan_array(const int32_t* in, int32_t* out, int n, uint32_
 template <class T, int D, bool IS_Q>
 __global__ void __launch_bounds__(kMergeThreads)
 merge_kernel(Dims dims, const BlockDesc* __restrict__ blocks, const T* __restrict__ X,
-             const T* __restrict__ V, Buffers buf, Debug dbg, int injected, int sortN) {
-  using Row = WarpRow<T, D>;
-  constexpr int E = Row::E;
+             const T* __restrict__ V, Buffers buf, Debug dbg, int injected, int cap) {
+  // shared memory: cap >= sources of any block (a multiple of the block size)
   extern __shared__ __align__(16) unsigned char smem[];
-  unsigned long long* keys = reinterpret_cast<unsigned long long*>(smem);
-  int32_t* cnt = reinterpret_cast<int32_t*>(keys + sortN);
-  int32_t* gst = cnt + dims.max_ndst;
-  uint32_t* hist = reinterpret_cast<uint32_t*>(gst + dims.max_ndst);
-  uint32_t* tmp = hist + (IS_Q ? kHistBins : 0);
+  uint32_t* key = reinterpret_cast<uint32_t*>(smem);        // [cap] ordered score bits
+  int32_t* mem = reinterpret_cast<int32_t*>(key + cap);      // [cap] merged by group, then kept
+  int32_t* aux = mem + cap;                                  // [cap] merged, unordered within a group
+  int32_t* cm = aux + cap;                                   // [max_ndst] merged sources per destination
+  int32_t* gsm = cm + dims.max_ndst;                         // [max_ndst] exclusive scan of cm
+  int32_t* cur = gsm + dims.max_ndst;                        // [max_ndst] placement cursors
+  uint32_t* rh = reinterpret_cast<uint32_t*>(cur + dims.max_ndst);  // [kHistBins] radix select
+  uint32_t* hist = rh + kHistBins;                           // [kHistBins] deviation keys (queries)
+  uint32_t* tmp = hist + kHistBins;                          // [64]
+  uint8_t* mf = reinterpret_cast<uint8_t*>(tmp + 64);        // [cap] merged flag
   __shared__ int s_bad;
   __shared__ uint32_t s_elig;
+  __shared__ int s_bin;
+  __shared__ uint32_t s_krem;
 
   const int tid = threadIdx.x, bd = blockDim.x;
   const int lane = tid & 31, warp = tid >> 5, nwarps = bd >> 5;
@@ -106,53 +191,123 @@ merge_kernel(Dims dims, const BlockDesc* __restrict__ blocks, const T* __restric
   const int slot_off = IS_Q ? b.q_slot_off : b.k_slot_off;
   const int nslots = IS_Q ? dims.q_slots : dims.k_slots;
   const size_t tokbase = (size_t)hh * dims.N;
+  // thread-contiguous source ranges for the order-dependent scans
+  const int per = (nsrc + bd - 1) / bd;
+  const int lo = min(nsrc, tid * per), hi = min(nsrc, lo + per);
 
   if (cta_plan_failed(buf.state)) return;
   if (tid == 0) { s_bad = 0; s_elig = 0; }
   if (IS_Q)
     for (int i = tid; i < kHistBins; i += bd) hist[i] = 0;
+  for (int m = tid; m < ndst; m += bd) cm[m] = 0;
 
-  // 1. top-r: the r sources with the largest (score, -ordinal) merge.
+  // 1. top-r: the r sources with the largest (score, -ordinal) merge.  The
+  //    r-th largest ordered score T comes from a 3-digit radix select; all
+  //    keys above T merge, and of the keys equal to T the lowest ordinals.
   if (!injected) {
-    for (int k = tid; k < sortN; k += bd)
-      keys[k] = k < nsrc ? ((unsigned long long)(~float_order(score[k])) << 32) | (unsigned)k : ~0ull;
-    __syncthreads();
-    block_bitonic_sort(keys, sortN);
-    for (int p = tid; p < nsrc; p += bd) merged[(uint32_t)keys[p]] = p < r ? 1 : 0;
-    __syncthreads();
+    for (int k = tid; k < nsrc; k += bd) key[k] = float_order(score[k]);
+    uint32_t T = 0, need = 0;
+    if (r > 0) {
+      uint32_t prefix = 0, krem = (uint32_t)r;
+#pragma unroll 1
+      for (int pass = 0; pass < 3; ++pass) {
+        const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+        const int nb = pass == 2 ? 1024 : 2048;
+        for (int i = tid; i < kHistBins; i += bd) rh[i] = 0;
+        __syncthreads();
+        for (int k = tid; k < nsrc; k += bd) {
+          const uint32_t kk = key[k];
+          if (pass == 0 || (kk >> (shift + (pass == 1 ? 11 : 10))) == prefix)
+            atomicAdd(&rh[(kk >> shift) & (uint32_t)(nb - 1)], 1u);
+        }
+        __syncthreads();
+        if (warp == 0) {
+          int bin;
+          uint32_t kr;
+          warp_select_bin(rh, nb, krem, &bin, &kr);
+          if (lane == 0) { s_bin = bin; s_krem = kr; }
+        }
+        __syncthreads();
+        prefix = (prefix << (pass == 2 ? 10 : 11)) | (uint32_t)s_bin;
+        krem = s_krem;
+      }
+      T = prefix;
+      need = krem;
+    }
+    uint32_t neq = 0;
+    for (int k = lo; k < hi; ++k) neq += r > 0 && key[k] == T;
+    uint32_t tot;
+    uint32_t eq_before = block_excl_scan(neq, tmp, &tot);
+    for (int k = lo; k < hi; ++k) {
+      bool m = false;
+      if (r > 0) {
+        const uint32_t kk = key[k];
+        m = kk > T || (kk == T && eq_before < need);
+        eq_before += kk == T;
+      }
+      mf[k] = m ? 1 : 0;
+      merged[k] = m ? 1 : 0;
+    }
   } else {
     uint32_t c = 0;
-    for (int k = tid; k < nsrc; k += bd) c += merged[k] != 0;
+    for (int k = tid; k < nsrc; k += bd) {
+      mf[k] = merged[k] != 0;
+      c += mf[k];
+    }
     uint32_t tot;
     block_excl_scan(c, tmp, &tot);
     if (tid == 0 && tot != (uint32_t)r) s_bad = 1;
   }
+  __syncthreads();
 
-  // 2. group members: (best destination, ordinal) for merged sources, kept
-  //    sources after them in ascending ordinal.
-  for (int k = tid; k < sortN; k += bd) {
-    unsigned long long v = ~0ull;
-    if (k < nsrc) {
-      if (merged[k]) {
-        int m = best[k];
-        if (m < 0 || m >= ndst) { s_bad = 1; m = 0; }
-        v = ((unsigned long long)m << 32) | (unsigned)k;
-      } else {
-        v = (0xFFFFFFFFull << 32) | (unsigned)k;
-      }
+  // 2. groups: merged sources per destination (counting), placement, then
+  //    each group's members put in ascending ordinal by rank counting (the
+  //    placement order of atomics is not deterministic, the ranks are).
+  for (int k = tid; k < nsrc; k += bd) {
+    if (mf[k]) {
+      const int m = best[k];
+      if (m < 0 || m >= ndst) s_bad = 1;
+      else atomicAdd(&cm[m], 1);
     }
-    keys[k] = v;
   }
-  for (int m = tid; m < ndst; m += bd) cnt[m] = 1;
   __syncthreads();
   if (s_bad) {
     if (tid == 0) set_status(buf.state, HTTM_DEV_BAD_PLAN);
     return;
   }
-  block_bitonic_sort(keys, sortN);
-  for (int p = tid; p < r; p += bd) atomicAdd(&cnt[keys[p] >> 32], 1);
+  block_scan_array(cm, gsm, ndst, tmp);
+  for (int m = tid; m < ndst; m += bd) cur[m] = gsm[m];
   __syncthreads();
-  block_scan_array(cnt, gst, ndst, tmp);
+  for (int k = tid; k < nsrc; k += bd)
+    if (mf[k]) aux[atomicAdd(&cur[best[k]], 1)] = k;
+  {
+    // kept sources in ascending ordinal after the r merged ones
+    uint32_t nm = 0;
+    for (int k = lo; k < hi; ++k) nm += mf[k];
+    uint32_t tot;
+    uint32_t before = block_excl_scan(nm, tmp, &tot);
+    for (int k = lo; k < hi; ++k) {
+      if (mf[k]) ++before;
+      else mem[r + (k - (int)before)] = k;
+    }
+  }
+  __syncthreads();
+  for (int m = warp; m < ndst; m += nwarps) {
+    const int s0 = gsm[m], c = cm[m];
+    for (int i = lane; i < c; i += 32) {
+      const int v = aux[s0 + i];
+      int rank = 0;
+      for (int j = 0; j < c; ++j) rank += aux[s0 + j] < v;
+      mem[s0 + rank] = v;
+    }
+  }
+  __syncthreads();
+  // original token of every member position, and of every destination
+  int32_t* tokm = aux;
+  int32_t* dtok = cur;
+  for (int x = tid; x < nsrc; x += bd) tokm[x] = block_token(b, src_index(mem[x], stride), dims.P);
+  for (int m = tid; m < ndst; m += bd) dtok[m] = block_token(b, m * stride, dims.P);
+  __syncthreads();
 
   const T* Xh = X + tokbase * D;
   const T* Vh = IS_Q ? nullptr : V + tokbase * D;
@@ -161,99 +316,137 @@ merge_kernel(Dims dims, const BlockDesc* __restrict__ blocks, const T* __restric
   float* dmean = IS_Q ? dbg.q_means : dbg.k_means;
   uint32_t elig = 0;
 
-  // 3. destination groups: mean of members; queries also get deviations.
-  for (int m = warp; m < ndst; m += nwarps) {
-    const int c = cnt[m];
-    const int ms = gst[m] - m;  // first merged member in keys[]
+  // 3. destination groups.  Rows are read as 16-byte chunks: lane l owns
+  //    chunk l % CPR, and the RPI row groups of a warp (CPR lanes each) work
+  //    on RPI different destination groups at once, each fetching up to kU
+  //    member rows before summing them -- up to RPI * kU rows in flight per
+  //    warp.  Members are summed in member order (destination first, then
+  //    merged sources by ascending in-block index); a member's deviation is
+  //    reduced over the CPR lanes of its row group.
+  using Ch = Chunk<T, D>;
+  constexpr int CPR = Ch::CPR, RPI = Ch::RPI, EPC = Ch::EPC, kU = 8;
+  const int rg = lane / CPR, ch = lane % CPR;
+  for (int m0 = warp * RPI; m0 < ndst; m0 += nwarps * RPI) {
+    const int m = m0 + rg;
+    const bool live = m < ndst;
+    const int c = live ? cm[m] + 1 : 0;    // members: the destination and its merged sources
+    const int cmax = __reduce_max_sync(0xffffffffu, c);
+    const int ms = live ? gsm[m] : 0;      // first merged member in mem[]
     const int slot = slot_off + m;
-    float acc[E], accv[E], x[E];
-    const int tok0 = block_token(b, m * stride, dims.P);
-    Row::load(Xh + (size_t)tok0 * D, lane, acc);
-    if (!IS_Q) Row::load(Vh + (size_t)tok0 * D, lane, accv);
-    for (int q = 0; q < c - 1; ++q) {
-      const int tok = block_token(b, src_index((int)(uint32_t)keys[ms + q], stride), dims.P);
-      Row::load(Xh + (size_t)tok * D, lane, x);
+    const int tok0 = live ? dtok[m] : 0;
+    auto member = [&](int q) -> int { return q == 0 ? tok0 : tokm[ms + q - 1]; };
+    float acc[EPC], accv[EPC];
 #pragma unroll
-      for (int e = 0; e < E; ++e) acc[e] += x[e];
-      if (!IS_Q) {
-        Row::load(Vh + (size_t)tok * D, lane, x);
+    for (int e = 0; e < EPC; ++e) acc[e] = accv[e] = 0.f;
+    uint4 xk[kU];                  // the first kU member chunks, kept for the deviations
+    for (int q0 = 0; q0 < cmax; q0 += kU) {
+      uint4 x[kU], xv[kU];
 #pragma unroll
-        for (int e = 0; e < E; ++e) accv[e] += x[e];
+      for (int u = 0; u < kU; ++u) {
+        if (q0 + u < c) {
+          const size_t off = (size_t)member(q0 + u) * D;
+          x[u] = Ch::load(Xh + off, ch);
+          if (!IS_Q) xv[u] = Ch::load(Vh + off, ch);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        if (q0 + u < c) {
+          Ch::add(acc, x[u]);
+          if (!IS_Q) Ch::add(accv, xv[u]);
+        }
+      }
+      if (q0 == 0) {
+#pragma unroll
+        for (int u = 0; u < kU; ++u) xk[u] = x[u];
       }
     }
-    const float fc = (float)c;
+    if (live) {
+      const float fc = (float)c;
 #pragma unroll
-    for (int e = 0; e < E; ++e) acc[e] = acc[e] / fc;
-    Row::store(Xt + (size_t)slot * D, lane, acc);
-    if (dmean) store_f32<E>(dmean + ((size_t)hh * nslots + slot) * D, lane, D, acc);
-    if (!IS_Q) {
-#pragma unroll
-      for (int e = 0; e < E; ++e) accv[e] = accv[e] / fc;
-      Row::store(Vt + (size_t)slot * D, lane, accv);
-      if (dbg.v_means) store_f32<E>(dbg.v_means + ((size_t)hh * nslots + slot) * D, lane, D, accv);
+      for (int e = 0; e < EPC; ++e) {
+        acc[e] = acc[e] / fc;
+        accv[e] = accv[e] / fc;
+      }
+      Ch::store(Xt + (size_t)slot * D, ch, acc);
+      if (dmean) Ch::store_f32(dmean + ((size_t)hh * nslots + slot) * D, ch, acc);
+      if (!IS_Q) {
+        Ch::store(Vt + (size_t)slot * D, ch, accv);
+        if (dbg.v_means) Ch::store_f32(dbg.v_means + ((size_t)hh * nslots + slot) * D, ch, accv);
+      }
     }
-    const int pos = b.tok_off + gst[m];
-    if (IS_Q && lane == 0) {
+    const int pos = live ? b.tok_off + gsm[m] + m : 0;
+    if (IS_Q && live && ch == 0) {
       buf.q_gstart[(size_t)hh * nslots + slot] = pos;
       buf.q_gcount[(size_t)hh * nslots + slot] = c;
     }
-    for (int q = 0; q < c; ++q) {
-      const int tok = q == 0 ? tok0
-                             : block_token(b, src_index((int)(uint32_t)keys[ms + q - 1], stride), dims.P);
-      if (IS_Q) {
-        uint32_t key = 0;
-        if (c >= 2) {
-          Row::load(Xh + (size_t)tok * D, lane, x);
-          float ss = 0.f;
+    for (int q0 = 0; q0 < cmax; q0 += kU) {
 #pragma unroll
-          for (int e = 0; e < E; ++e) {
-            const float df = x[e] - acc[e];
-            ss = fmaf(df, df, ss);
+      for (int u = 0; u < kU; ++u) {
+        const int q = q0 + u;
+        const bool mine = q < c;
+        const int tok = mine ? member(q) : 0;
+        if (IS_Q) {
+          uint4 xr = xk[u];
+          if (q0 > 0 && mine && c >= 2) xr = Ch::load(Xh + (size_t)tok * D, ch);
+          const float ss = Ch::within_row(mine ? Ch::sq_dist(xr, acc) : 0.f);
+          if (mine && ch == 0) {
+            const uint32_t key = c >= 2 ? __float_as_uint(sqrtf(ss)) + 1u : 0u;
+            buf.q_members[tokbase + pos + q] = tok;
+            buf.q_slot[tokbase + tok] = slot;
+            buf.keys[tokbase + tok] = key;
+            if (key) {
+              atomicAdd(&hist[key >> 21], 1u);
+              ++elig;
+            }
           }
-          ss = warp_sum(ss);
-          key = __float_as_uint(sqrtf(ss)) + 1u;
+        } else if (mine && dbg.k_slot && ch == 0) {
+          dbg.k_slot[tokbase + tok] = slot;
         }
-        if (lane == 0) {
-          buf.q_members[tokbase + pos + q] = tok;
-          buf.q_slot[tokbase + tok] = slot;
-          buf.keys[tokbase + tok] = key;
-          if (key) {
-            atomicAdd(&hist[key >> 21], 1u);
-            ++elig;
-          }
-        }
-      } else if (dbg.k_slot && lane == 0) {
-        dbg.k_slot[tokbase + tok] = slot;
       }
     }
   }
 
-  // 4. kept sources: singleton slots after the destination groups.
-  for (int p = r + warp; p < nsrc; p += nwarps) {
-    const int rank = p - r;
-    const int slot = slot_off + ndst + rank;
-    const int tok = block_token(b, src_index((int)(uint32_t)keys[p], stride), dims.P);
-    float x[E];
-    Row::load(Xh + (size_t)tok * D, lane, x);
-    Row::store(Xt + (size_t)slot * D, lane, x);
-    if (dmean) store_f32<E>(dmean + ((size_t)hh * nslots + slot) * D, lane, D, x);
-    if (!IS_Q) {
-      Row::load(Vh + (size_t)tok * D, lane, x);
-      Row::store(Vt + (size_t)slot * D, lane, x);
-      if (dbg.v_means) store_f32<E>(dbg.v_means + ((size_t)hh * nslots + slot) * D, lane, D, x);
-      if (dbg.k_slot && lane == 0) dbg.k_slot[tokbase + tok] = slot;
-    } else if (lane == 0) {
-      const int pos = b.tok_off + ndst + r + rank;
-      buf.q_members[tokbase + pos] = tok;
-      buf.q_slot[tokbase + tok] = slot;
-      buf.keys[tokbase + tok] = 0u;
-      buf.q_gstart[(size_t)hh * nslots + slot] = pos;
-      buf.q_gcount[(size_t)hh * nslots + slot] = 1;
+  // 4. kept sources: singleton slots after the destination groups, copied
+  //    RPI * kU rows per warp step.
+  for (int p0 = r + warp * RPI * kU; p0 < nsrc; p0 += nwarps * RPI * kU) {
+    uint4 x[kU], xv[kU];
+    int tk[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int p = p0 + rg + RPI * u;
+      tk[u] = p < nsrc ? tokm[p] : 0;
+      if (p < nsrc) {
+        x[u] = Ch::load(Xh + (size_t)tk[u] * D, ch);
+        if (!IS_Q) xv[u] = Ch::load(Vh + (size_t)tk[u] * D, ch);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int p = p0 + rg + RPI * u;
+      if (p >= nsrc) continue;
+      const int rank = p - r;
+      const int slot = slot_off + ndst + rank;
+      const int tok = tk[u];
+      Ch::store_raw(Xt + (size_t)slot * D, ch, x[u]);
+      if (dmean) Ch::store_raw_f32(dmean + ((size_t)hh * nslots + slot) * D, ch, x[u]);
+      if (!IS_Q) {
+        Ch::store_raw(Vt + (size_t)slot * D, ch, xv[u]);
+        if (dbg.v_means) Ch::store_raw_f32(dbg.v_means + ((size_t)hh * nslots + slot) * D, ch, xv[u]);
+        if (dbg.k_slot && ch == 0) dbg.k_slot[tokbase + tok] = slot;
+      } else if (ch == 0) {
+        const int pos = b.tok_off + ndst + r + rank;
+        buf.q_members[tokbase + pos] = tok;
+        buf.q_slot[tokbase + tok] = slot;
+        buf.keys[tokbase + tok] = 0u;
+        buf.q_gstart[(size_t)hh * nslots + slot] = pos;
+        buf.q_gcount[(size_t)hh * nslots + slot] = 1;
+      }
     }
   }
 
   if (IS_Q) {
-    if (lane == 0 && elig) atomicAdd(&s_elig, elig);
+    if (elig) atomicAdd(&s_elig, elig);
     __syncthreads();
     for (int i = tid; i < kHistBins; i += bd)
       if (hist[i]) atomicAdd(&buf.hist[i], hist[i]);
@@ -422,17 +615,18 @@ template <class T, int D>
 cudaError_t launch_merge_t(const Dims& dims, const BlockDesc* blocks, bool is_q, bool injected,
                            const void* X, const void* V, const Buffers& buf, const Debug& dbg,
                            cudaStream_t s) {
-  const int sortN = next_pow2(dims.max_nsrc);
-  const size_t smem = (size_t)sortN * 8 + 2ull * dims.max_ndst * 4 + (is_q ? kHistBins * 4 : 0) + 64 * 4;
+  const int cap = (dims.max_nsrc + kMergeThreads - 1) / kMergeThreads * kMergeThreads;
+  const size_t smem = (size_t)cap * 13 + 3ull * dims.max_ndst * 4 + 2ull * kHistBins * 4 + 64 * 4;
   dim3 grid(dims.nblk, dims.h);
+  cudaError_t e;
   if (is_q) {
     auto k = merge_kernel<T, D, true>;
-    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    k<<<grid, kMergeThreads, smem, s>>>(dims, blocks, (const T*)X, nullptr, buf, dbg, injected, sortN);
+    if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e;
+    k<<<grid, kMergeThreads, smem, s>>>(dims, blocks, (const T*)X, nullptr, buf, dbg, injected, cap);
   } else {
     auto k = merge_kernel<T, D, false>;
-    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    k<<<grid, kMergeThreads, smem, s>>>(dims, blocks, (const T*)X, (const T*)V, buf, dbg, injected, sortN);
+    if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e;
+    k<<<grid, kMergeThreads, smem, s>>>(dims, blocks, (const T*)X, (const T*)V, buf, dbg, injected, cap);
   }
   return cudaGetLastError();
 }
