@@ -11,21 +11,24 @@
 //   warp 0      TMA producer: both Q tiles once, then K/V tiles of 128 keys
 //               into a 4-stage shared-memory ring;
 //   warp 1      one thread issues tcgen05.mma:
-//                 S_t = Q_t K_j^T   (M=128, N=128, K=64; A, B in shared memory)
-//                 O_t += P_t V_j    (M=128, N=64, K=128; A = P_t in TMEM)
-//               in the order  PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1);
+//                 S = Q_t K_j^T     (M=128, N=128, K=64; A, B in shared memory)
+//                 O_t += P V_j      (M=128, N=64, K=128; A = P in TMEM)
+//               in the order  PV(0,j), QK(1,j+1), PV(1,j), QK(0,j+2);
 //   warps 2, 3  idle;
 //   warps 4..7  softmax of tile 0, warps 8..11 softmax of tile 1: one query
 //               row per thread (TMEM lane = row).
 // Registers: launched at 168 per thread (384 x 168 = 64,512); warpgroup 0
 // gives part of its share back (setmaxnreg to 88) and the softmax warpgroups
 // take it (208): 128 x 88 + 256 x 208 = 64,512.
-// TMEM (512 columns): per tile t, S_t [t*256, +128), P_t [t*256+128, +64)
-// (bf16 pairs), O_t [t*256+192, +64).  Tensor-core operations complete in
-// issue order, so when S_t(j+1) is ready, PV_t(j) -- the last reader of P_t
-// and the last writer of O_t -- is done: the softmax may overwrite P_t and
-// rescale O_t without a further wait.  Two warpgroups keep two softmax warps
-// per SM sub-partition busy on the exp unit while the tensor core alternates
+// TMEM (512 columns): a ring of three 128-column S buffers [0, 384) -- the
+// i-th S product, i = 2j + t, goes to buffer i % 3, and the softmax writes
+// that tile's P (bf16 pairs, 64 columns) over the first half of the same
+// buffer once S is in registers -- then O_0 [384, 448) and O_1 [448, 512).
+// Tensor-core operations complete in issue order: S product i + 3 reuses a
+// buffer only after the PV that read P from it, and a softmax sees S for
+// (0, j+1) before it finishes (0, j).  A softmax that rescales O_t waits for
+// PV(t, j-1) first.  Two warpgroups keep two softmax warps per SM
+// sub-partition busy on the exp unit while the tensor core alternates
 // between the tiles.
 //
 // Softmax: base-2 running max, updated lazily -- O_t and the row sum are
@@ -51,7 +54,7 @@ constexpr int kD = 64;
 constexpr int kStages = 4;
 constexpr int kThreads = 384;
 constexpr uint32_t kTile = kBN * kD * 2;   // 16 KB: 128 rows x 64 bf16
-constexpr uint32_t kColS = 0, kColP = 128, kColO = 192, kColTile = 256;
+constexpr uint32_t kColO = 384;             // O_t at kColO + 64 t; S ring buffers at 0, 128, 256
 
 struct AttnSmem {
   uint8_t q[2][kTile];
@@ -59,7 +62,7 @@ struct AttnSmem {
   uint8_t v[kStages][kTile];
   uint64_t q_full;
   uint64_t kv_full[kStages], kv_empty[kStages];
-  uint64_t s_full[2], p_full[2], o_done[2];
+  uint64_t s_full[3], p_full[2], o_done[2];
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -96,8 +99,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
       mbar_init(&sm.kv_full[s], 1);
       mbar_init(&sm.kv_empty[s], 1);
     }
+    for (int i = 0; i < 3; ++i) mbar_init(&sm.s_full[i], 1);
     for (int t = 0; t < 2; ++t) {
-      mbar_init(&sm.s_full[t], 1);
       mbar_init(&sm.p_full[t], 128);
       mbar_init(&sm.o_done[t], 1);
     }
@@ -132,39 +135,49 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
       // ------------------------------------------------------------ MMA issue
       constexpr uint32_t id_s = idesc_bf16(kBM, kBN, false, false);
       constexpr uint32_t id_o = idesc_bf16(kBM, kD, false, true);
+      // S product i = 2j + t into ring buffer i % 3
       auto issue_qk = [&](int t, int j) {
         const uint32_t q_addr = smem_u32(sm.q[t]);
         const uint32_t k_addr = smem_u32(sm.k[j % kStages]);
+        const int bsel = (2 * j + t) % 3;
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk)
-          umma_bf16(tmem + t * kColTile + kColS, sw128_desc(q_addr + kk * 32, 1024),
-                    sw128_desc(k_addr + kk * 32, 1024), id_s, kk > 0);
-        umma_commit(&sm.s_full[t]);
+          umma_bf16(tmem + bsel * kBN, sw128_desc(q_addr + kk * 32, 1024), sw128_desc(k_addr + kk * 32, 1024),
+                    id_s, kk > 0);
+        umma_commit(&sm.s_full[bsel]);
       };
       auto issue_pv = [&](int t, int j) {
         const uint32_t v_addr = smem_u32(sm.v[j % kStages]);
+        const uint32_t p_col = (uint32_t)((2 * j + t) % 3) * kBN;
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk)
-          umma_bf16_ts(tmem + t * kColTile + kColO, tmem + t * kColTile + kColP + kk * 8,
-                       sw128_desc(v_addr + kk * 16 * 128, 1024), id_o, (j > 0 || kk > 0) ? 1u : 0u);
+          umma_bf16_ts(tmem + kColO + t * kD, tmem + p_col + kk * 8, sw128_desc(v_addr + kk * 16 * 128, 1024), id_o,
+                       (j > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(&sm.o_done[t]);
       };
       bool ok = mbar_wait(&sm.q_full, 0, abort, st) && mbar_wait(&sm.kv_full[0], 0, abort, st);
       if (ok) {
         tc_fence_after();
         issue_qk(0, 0);
         issue_qk(1, 0);
+        if (n_kv > 1) {
+          ok = mbar_wait(&sm.kv_full[1 % kStages], (1 / kStages) & 1, abort, st);
+          if (ok) issue_qk(0, 1);
+        }
       }
       for (int j = 0; ok && j < n_kv; ++j) {
-        const bool more = j + 1 < n_kv;
-        if (more && !mbar_wait(&sm.kv_full[(j + 1) % kStages], ((j + 1) / kStages) & 1, abort, st)) break;
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          if (!mbar_wait(&sm.p_full[t], j & 1, abort, st)) { ok = false; break; }
+        if (!mbar_wait(&sm.p_full[0], j & 1, abort, st)) break;
+        tc_fence_after();
+        issue_pv(0, j);
+        if (j + 1 < n_kv) issue_qk(1, j + 1);          // K_{j+1} arrived before QK(0, j+1)
+        if (!mbar_wait(&sm.p_full[1], j & 1, abort, st)) break;
+        tc_fence_after();
+        issue_pv(1, j);
+        umma_commit(&sm.kv_empty[j % kStages]);
+        if (j + 2 < n_kv) {
+          if (!mbar_wait(&sm.kv_full[(j + 2) % kStages], ((j + 2) / kStages) & 1, abort, st)) break;
           tc_fence_after();
-          issue_pv(t, j);
-          if (t == 1) umma_commit(&sm.kv_empty[j % kStages]);
-          if (more) issue_qk(t, j + 1);
-          else umma_commit(&sm.o_done[t]);
+          issue_qk(0, j + 2);
         }
       }
       // every MMA issued above completes before TMEM is released
@@ -178,17 +191,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;                // row inside the tile = TMEM lane
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    const uint32_t ts = tmem + lane_off + t * kColTile;
+    const uint32_t to = tmem + lane_off + kColO + t * kD;    // this row of O_t
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n_kv; ++j) {
+      const int qi = 2 * j + t, bsel = qi % 3;              // S product index and its ring buffer
+      const uint32_t ts = tmem + lane_off + bsel * kBN;    // this row of S, then of P
       // waits are made warp-uniform: tcgen05.ld/st below need every lane
-      if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[t], j & 1, abort, st))) { ok = false; break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[bsel], (qi / 3) & 1, abort, st))) { ok = false; break; }
       tc_fence_after();
       uint32_t sr[128];
 #pragma unroll
       for (int c = 0; c < 4; ++c)
-        tmem_ld32(ts + kColS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+        tmem_ld32(ts + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
       tmem_wait_ld();
       const int valid = Lk - j * kBN;
       if (valid < kBN) {
@@ -209,15 +224,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         const float m_new = fmaxf(m_used, mts);
         const float alpha = ex2(m_used - m_new);
         if (j > 0) {
-          // PV_t(j-1) completed before S_t(j) was signalled
+          if (!__all_sync(0xffffffffu, mbar_wait(&sm.o_done[t], (j - 1) & 1, abort, st))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
             uint32_t o[32];
-            tmem_ld32(ts + kColO + c * 32, o);
+            tmem_ld32(to + c * 32, o);
             tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st32(ts + kColO + c * 32, o);
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(to + c * 32, o);
           }
         }
         l *= alpha;
@@ -238,21 +257,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
           rs[(2 * i + 1) & 7] += p1;
           pk[i] = pack_bf16(p0, p1);
         }
-        tmem_st32(ts + kColP + c * 32, pk);
+        tmem_st32(ts + c * 32, pk);
       }
       l += ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&sm.p_full[t]);
     }
-    if (ok && __all_sync(0xffffffffu, mbar_wait(&sm.o_done[t], 0, abort, st))) {
+    if (ok && __all_sync(0xffffffffu, mbar_wait(&sm.o_done[t], (n_kv - 1) & 1, abort, st))) {
       tc_fence_after();
       const float inv = 1.f / l;
       uint32_t packed[32];
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t o[32];
-        tmem_ld32(ts + kColO + c * 32, o);
+        tmem_ld32(to + c * 32, o);
         tmem_wait_ld();
 #pragma unroll
         for (int i = 0; i < 16; ++i)
