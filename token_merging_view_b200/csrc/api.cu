@@ -110,6 +110,9 @@ Workspace layout(const Dims& d, bool fp32) {
   w.q_members = take(hN * 4);
   w.q_gstart = take((size_t)d.h * d.q_slots * 4);
   w.q_gcount = take((size_t)d.h * d.q_slots * 4);
+  w.k_members = take(hN * 4);
+  w.k_gstart = take((size_t)d.h * d.k_slots * 4);
+  w.k_gcount = take((size_t)d.h * d.k_slots * 4);
   w.q_tilde = take((size_t)d.q_rows_alloc * d.d * es);
   w.k_tilde = take((size_t)d.h * d.k_slots * d.d * es);
   w.v_tilde = take((size_t)d.h * d.k_slots * d.d * es);
@@ -139,6 +142,9 @@ Buffers resolve(const Workspace& w, void* base) {
   b.q_members = reinterpret_cast<int32_t*>(p + w.q_members);
   b.q_gstart = reinterpret_cast<int32_t*>(p + w.q_gstart);
   b.q_gcount = reinterpret_cast<int32_t*>(p + w.q_gcount);
+  b.k_members = reinterpret_cast<int32_t*>(p + w.k_members);
+  b.k_gstart = reinterpret_cast<int32_t*>(p + w.k_gstart);
+  b.k_gcount = reinterpret_cast<int32_t*>(p + w.k_gcount);
   b.q_tilde = p + w.q_tilde;
   b.k_tilde = p + w.k_tilde;
   b.v_tilde = p + w.v_tilde;
@@ -253,9 +259,9 @@ httm_status forward_impl(httm_plan_s* plan, const void* Q, const void* K, const 
     if (e != cudaSuccess) return HTTM_ERR_CUDA;
   }
   {
-    StageTimer t(plan, s, HTTM_STAGE_MERGE, 2);
-    HTTM_LAUNCH(launch_merge(dims, fp32, plan->blocks_d, true, plan_inj, Q, nullptr, buf, dd, s));
-    HTTM_LAUNCH(launch_merge(dims, fp32, plan->blocks_d, false, plan_inj, K, V, buf, dd, s));
+    StageTimer t(plan, s, HTTM_STAGE_MERGE, 3);
+    HTTM_LAUNCH(launch_merge(dims, fp32, plan->blocks_d, plan_inj, Q, K, V, buf, dd, s));
+    launches += 2;  // planning, then the two gathers
   }
   {
     StageTimer t(plan, s, HTTM_STAGE_OUTLIER, mask_inj ? 4 : 6);

@@ -211,13 +211,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         for (int i = 0; i < kBN; ++i)
           if (i >= valid) sr[i] = __float_as_uint(-INFINITY);
       }
-      float mx[8];
+      // row max: four chains of three-input max
+      float mx[4];
 #pragma unroll
-      for (int a = 0; a < 8; ++a) mx[a] = __uint_as_float(sr[a]);
+      for (int a = 0; a < 4; ++a) mx[a] = __uint_as_float(sr[a]);
 #pragma unroll
-      for (int i = 8; i < kBN; ++i) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(sr[i]));
-      const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      for (int i = 4; i < kBN; i += 8) {
+#pragma unroll
+        for (int a = 0; a < 4; ++a) mx[a] = max3(mx[a], __uint_as_float(sr[i + a]), __uint_as_float(sr[i + 4 + a]));
+      }
+      const float mt = max3(mx[0], mx[1], fmaxf(mx[2], mx[3]));
       const float mts = mt * scale_log2;
       const bool need = mts > m_used + 8.f;
       if (__any_sync(0xffffffffu, need)) {
@@ -242,24 +245,34 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         l *= alpha;
         m_used = m_new;
       }
-      const float neg_m = -m_used;
-      float rs[8];
+      // p = 2^(s * c - m): the affine part and the row sums on packed fp32
+      // pairs, the exponentials on the exp unit
+      const unsigned long long cc = f2_pack(scale_log2, scale_log2);
+      const unsigned long long mm = f2_pack(-m_used, -m_used);
+      unsigned long long rs[4];
 #pragma unroll
-      for (int a = 0; a < 8; ++a) rs[a] = 0.f;
+      for (int a = 0; a < 4; ++a) rs[a] = 0ull;           // (0.f, 0.f)
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t pk[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const float p0 = ex2(fmaf(__uint_as_float(sr[c * 64 + 2 * i]), scale_log2, neg_m));
-          const float p1 = ex2(fmaf(__uint_as_float(sr[c * 64 + 2 * i + 1]), scale_log2, neg_m));
-          rs[(2 * i) & 7] += p0;
-          rs[(2 * i + 1) & 7] += p1;
+          const unsigned long long xp =
+              f2_fma(f2_pack(__uint_as_float(sr[c * 64 + 2 * i]), __uint_as_float(sr[c * 64 + 2 * i + 1])), cc, mm);
+          float x0, x1;
+          f2_unpack(xp, x0, x1);
+          const float p0 = ex2(x0), p1 = ex2(x1);
+          rs[i & 3] = f2_add(rs[i & 3], f2_pack(p0, p1));
           pk[i] = pack_bf16(p0, p1);
         }
         tmem_st32(ts + c * 32, pk);
       }
-      l += ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
+      float r0, r1, r2, r3, r4, r5, r6, r7;
+      f2_unpack(rs[0], r0, r1);
+      f2_unpack(rs[1], r2, r3);
+      f2_unpack(rs[2], r4, r5);
+      f2_unpack(rs[3], r6, r7);
+      l += ((r0 + r1) + (r2 + r3)) + ((r4 + r5) + (r6 + r7));
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&sm.p_full[t]);

@@ -55,7 +55,7 @@ struct DevState {
 struct Workspace {
   size_t state, hist, chunk, n_out, out_base, items;
   size_t q_best, q_score, q_merged, k_best, k_score, k_merged;
-  size_t q_slot, keys, mask, q_members, q_gstart, q_gcount;
+  size_t q_slot, keys, mask, q_members, q_gstart, q_gcount, k_members, k_gstart, k_gcount;
   size_t q_tilde, k_tilde, v_tilde, o_tilde;
   size_t total;
 };
@@ -75,9 +75,12 @@ struct Buffers {
   int32_t* q_slot;         // [h, N]
   uint32_t* keys;          // [h, N]: eligible ? bits(dev) + 1 : 0
   uint8_t* mask;           // [h, N]
-  int32_t* q_members;      // [h, N]: tokens in group order, per block
-  int32_t* q_gstart;       // [h, q_slots]: first member position (dst groups)
-  int32_t* q_gcount;       // [h, q_slots]
+  int32_t* q_members;      // [h, N]: tokens in slot order (block after block)
+  int32_t* q_gstart;       // [h, q_slots]: first member position of each slot
+  int32_t* q_gcount;       // [h, q_slots]: members of each slot
+  int32_t* k_members;      // the same for the key plan (values follow it)
+  int32_t* k_gstart;
+  int32_t* k_gcount;
   void* q_tilde; void* k_tilde; void* v_tilde; void* o_tilde;
 };
 

@@ -36,8 +36,10 @@ cudaError_t launch_match_tc(const Dims& dims, const BlockDesc* blocks, const int
 cudaError_t launch_import_plan(const Dims& dims, const BlockDesc* blocks, const Inject& inj,
                                const Buffers& buf, cudaStream_t s);
 
-cudaError_t launch_merge(const Dims& dims, bool fp32, const BlockDesc* blocks, bool is_q,
-                         bool injected, const void* X, const void* V, const Buffers& buf,
+// Merge planning (Q and K) then the mean-merging gathers of Q and of K/V:
+// three launches.
+cudaError_t launch_merge(const Dims& dims, bool fp32, const BlockDesc* blocks, bool injected,
+                         const void* Q, const void* K, const void* V, const Buffers& buf,
                          const Debug& dbg, cudaStream_t s);
 
 cudaError_t launch_outlier(const Dims& dims, bool fp32, const void* Q, bool mask_injected,

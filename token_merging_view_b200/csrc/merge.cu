@@ -155,11 +155,38 @@ __device__ void block_scan_array(const int32_t* in, int32_t* out, int n, uint32_
   __syncthreads();
 }
 
-template <class T, int D, bool IS_Q>
+// The bin holding the k-th largest element (k >= 1) of hist[0, nb) and k
+// minus the elements in higher bins, by the whole thread block: each thread
+// owns nb / blockDim.x consecutive bins from the top, one block scan finds
+// the owner.  Results land in *bin / *krem (shared memory).
+__device__ void block_select_bin(const uint32_t* hist, int nb, uint32_t k, uint32_t* tmp, int* bin, uint32_t* krem) {
+  const int per = nb / blockDim.x;
+  const int top = nb - 1 - threadIdx.x * per;
+  uint32_t s = 0;
+  for (int i = 0; i < per; ++i) s += hist[top - i];
+  uint32_t tot;
+  uint32_t above = block_excl_scan(s, tmp, &tot);
+  if (above < k && k <= above + s) {
+    for (int i = 0; i < per; ++i) {
+      const uint32_t c = hist[top - i];
+      if (k <= above + c) {
+        *bin = top - i;
+        *krem = k - above;
+        break;
+      }
+      above += c;
+    }
+  }
+  __syncthreads();
+}
+
+// Merge planning, one CTA per (block, head, tensor): which sources merge
+// (top-r), their groups, and the member lists (CSR) the gather kernel reads.
+// Members of a destination group: the destination, then its merged sources
+// by ascending in-block index; kept sources follow as singletons.  Every
+// token of the block is the member of exactly one slot.
 __global__ void __launch_bounds__(kMergeThreads)
-merge_kernel(Dims dims, const BlockDesc* __restrict__ blocks, const T* __restrict__ X,
-             const T* __restrict__ V, Buffers buf, Debug dbg, int injected, int cap) {
-  // shared memory: cap >= sources of any block (a multiple of the block size)
+plan_kernel(Dims dims, const BlockDesc* __restrict__ blocks, Buffers buf, Debug dbg, int injected, int cap) {
   extern __shared__ __align__(16) unsigned char smem[];
   uint32_t* key = reinterpret_cast<uint32_t*>(smem);        // [cap] ordered score bits
   int32_t* mem = reinterpret_cast<int32_t*>(key + cap);      // [cap] merged by group, then kept
@@ -168,37 +195,37 @@ merge_kernel(Dims dims, const BlockDesc* __restrict__ blocks, const T* __restric
   int32_t* gsm = cm + dims.max_ndst;                         // [max_ndst] exclusive scan of cm
   int32_t* cur = gsm + dims.max_ndst;                        // [max_ndst] placement cursors
   uint32_t* rh = reinterpret_cast<uint32_t*>(cur + dims.max_ndst);  // [kHistBins] radix select
-  uint32_t* hist = rh + kHistBins;                           // [kHistBins] deviation keys (queries)
-  uint32_t* tmp = hist + kHistBins;                          // [64]
+  uint32_t* tmp = rh + kHistBins;                            // [64]
   uint8_t* mf = reinterpret_cast<uint8_t*>(tmp + 64);        // [cap] merged flag
   __shared__ int s_bad;
-  __shared__ uint32_t s_elig;
   __shared__ int s_bin;
   __shared__ uint32_t s_krem;
 
+  const bool is_q = blockIdx.z == 0;
   const int tid = threadIdx.x, bd = blockDim.x;
   const int lane = tid & 31, warp = tid >> 5, nwarps = bd >> 5;
   const int hh = blockIdx.y;
   const BlockDesc b = blocks[blockIdx.x];
-  const int stride = IS_Q ? dims.q_stride : dims.kv_stride;
-  const int ndst = IS_Q ? b.q_ndst : b.k_ndst;
-  const int r = IS_Q ? b.q_r : b.k_r;
+  const int stride = is_q ? dims.q_stride : dims.kv_stride;
+  const int ndst = is_q ? b.q_ndst : b.k_ndst;
+  const int r = is_q ? b.q_r : b.k_r;
   const int nsrc = b.n_b - ndst;
-  const size_t sbase = (size_t)hh * (IS_Q ? dims.q_src : dims.k_src) + (IS_Q ? b.q_src_off : b.k_src_off);
-  const int32_t* best = (IS_Q ? buf.q_best : buf.k_best) + sbase;
-  const float* score = (IS_Q ? buf.q_score : buf.k_score) + sbase;
-  uint8_t* merged = (IS_Q ? buf.q_merged : buf.k_merged) + sbase;
-  const int slot_off = IS_Q ? b.q_slot_off : b.k_slot_off;
-  const int nslots = IS_Q ? dims.q_slots : dims.k_slots;
+  const size_t sbase = (size_t)hh * (is_q ? dims.q_src : dims.k_src) + (is_q ? b.q_src_off : b.k_src_off);
+  const int32_t* best = (is_q ? buf.q_best : buf.k_best) + sbase;
+  const float* score = (is_q ? buf.q_score : buf.k_score) + sbase;
+  uint8_t* merged = (is_q ? buf.q_merged : buf.k_merged) + sbase;
+  const int slot_off = is_q ? b.q_slot_off : b.k_slot_off;
+  const int nslots = is_q ? dims.q_slots : dims.k_slots;
   const size_t tokbase = (size_t)hh * dims.N;
+  int32_t* members = (is_q ? buf.q_members : buf.k_members) + tokbase;
+  int32_t* gstart = (is_q ? buf.q_gstart : buf.k_gstart) + (size_t)hh * nslots;
+  int32_t* gcount = (is_q ? buf.q_gcount : buf.k_gcount) + (size_t)hh * nslots;
   // thread-contiguous source ranges for the order-dependent scans
   const int per = (nsrc + bd - 1) / bd;
   const int lo = min(nsrc, tid * per), hi = min(nsrc, lo + per);
 
   if (cta_plan_failed(buf.state)) return;
-  if (tid == 0) { s_bad = 0; s_elig = 0; }
-  if (IS_Q)
-    for (int i = tid; i < kHistBins; i += bd) hist[i] = 0;
+  if (tid == 0) s_bad = 0;
   for (int m = tid; m < ndst; m += bd) cm[m] = 0;
 
   // 1. top-r: the r sources with the largest (score, -ordinal) merge.  The
@@ -221,13 +248,7 @@ merge_kernel(Dims dims, const BlockDesc* __restrict__ blocks, const T* __restric
             atomicAdd(&rh[(kk >> shift) & (uint32_t)(nb - 1)], 1u);
         }
         __syncthreads();
-        if (warp == 0) {
-          int bin;
-          uint32_t kr;
-          warp_select_bin(rh, nb, krem, &bin, &kr);
-          if (lane == 0) { s_bin = bin; s_krem = kr; }
-        }
-        __syncthreads();
+        block_select_bin(rh, nb, krem, tmp, &s_bin, &s_krem);
         prefix = (prefix << (pass == 2 ? 10 : 11)) | (uint32_t)s_bin;
         krem = s_krem;
       }
@@ -292,8 +313,23 @@ merge_kernel(Dims dims, const BlockDesc* __restrict__ blocks, const T* __restric
     }
   }
   __syncthreads();
+  // small groups: one thread, insertion order; large groups: one warp, ranks
+  for (int m = tid; m < ndst; m += bd) {
+    const int s0 = gsm[m], c = cm[m];
+    if (c > 32) continue;
+    for (int i = 0; i < c; ++i) {
+      const int v = aux[s0 + i];
+      int j = i;
+      while (j > 0 && mem[s0 + j - 1] > v) {
+        mem[s0 + j] = mem[s0 + j - 1];
+        --j;
+      }
+      mem[s0 + j] = v;
+    }
+  }
   for (int m = warp; m < ndst; m += nwarps) {
     const int s0 = gsm[m], c = cm[m];
+    if (c <= 32) continue;
     for (int i = lane; i < c; i += 32) {
       const int v = aux[s0 + i];
       int rank = 0;
@@ -302,215 +338,255 @@ merge_kernel(Dims dims, const BlockDesc* __restrict__ blocks, const T* __restric
     }
   }
   __syncthreads();
-  // original token of every member position, and of every destination
-  int32_t* tokm = aux;
-  int32_t* dtok = cur;
-  for (int x = tid; x < nsrc; x += bd) tokm[x] = block_token(b, src_index(mem[x], stride), dims.P);
-  for (int m = tid; m < ndst; m += bd) dtok[m] = block_token(b, m * stride, dims.P);
-  __syncthreads();
 
-  const T* Xh = X + tokbase * D;
-  const T* Vh = IS_Q ? nullptr : V + tokbase * D;
-  T* Xt = reinterpret_cast<T*>(IS_Q ? buf.q_tilde : buf.k_tilde) + (size_t)hh * nslots * D;
-  T* Vt = IS_Q ? nullptr : reinterpret_cast<T*>(buf.v_tilde) + (size_t)hh * nslots * D;
+  // 3. member lists (tokens), slot starts and counts, the query slot map
+  for (int m = tid; m < ndst; m += bd) {
+    const int slot = slot_off + m;
+    const int pos = b.tok_off + gsm[m] + m;
+    const int c = cm[m] + 1;
+    for (int q = 0; q < c; ++q) {
+      const int tok = q == 0 ? block_token(b, m * stride, dims.P)
+                             : block_token(b, src_index(mem[gsm[m] + q - 1], stride), dims.P);
+      members[pos + q] = tok;
+      if (is_q) buf.q_slot[tokbase + tok] = slot;
+      else if (dbg.k_slot) dbg.k_slot[tokbase + tok] = slot;
+    }
+    gstart[slot] = pos;
+    gcount[slot] = c;
+  }
+  for (int p = tid; p < nsrc - r; p += bd) {
+    const int slot = slot_off + ndst + p;
+    const int pos = b.tok_off + ndst + r + p;
+    const int tok = block_token(b, src_index(mem[r + p], stride), dims.P);
+    members[pos] = tok;
+    gstart[slot] = pos;
+    gcount[slot] = 1;
+    if (is_q) buf.q_slot[tokbase + tok] = slot;
+    else if (dbg.k_slot) dbg.k_slot[tokbase + tok] = slot;
+  }
+}
+
+// Mean merging (key design 1), flat over every (head, slot).  Rows are read
+// as 16-byte chunks, lane l owning chunk l % CPR; each of the RPI row groups
+// of a warp (CPR lanes) takes its own slot, fetches up to kU member rows
+// before summing them in member order, and meanwhile already fetches the
+// (start, count) and first member indices of its next slot, so the CSR
+// lookups overlap the row loads.  Queries also get each member's deviation
+// from the mean (key design 3), kept as a 32-bit key (bits(dev) + 1 for
+// members of groups of >= 2, else 0), and the first radix digit of those
+// keys is histogrammed for the global outlier select.
+template <class T, int D, bool IS_Q>
+__global__ void __launch_bounds__(256)
+gather_kernel(Dims dims, const T* __restrict__ X, const T* __restrict__ V, Buffers buf, Debug dbg) {
+  using Ch = Chunk<T, D>;
+  constexpr int CPR = Ch::CPR, RPI = Ch::RPI, EPC = Ch::EPC, kU = 4;
+  __shared__ uint32_t hist[IS_Q ? kHistBins : 1];
+  __shared__ uint32_t s_elig;
+  if (cta_plan_failed(buf.state)) return;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int rg = lane / CPR, ch = lane % CPR;
+  if (IS_Q) {
+    for (int i = tid; i < kHistBins; i += blockDim.x) hist[i] = 0;
+    if (tid == 0) s_elig = 0;
+    __syncthreads();
+  }
+  // (head, slot) pairs are numbered gsl = head * nslots + slot; the plan
+  // limits h * N to 2^31 - 1, so 32-bit indices suffice
+  const int nslots = IS_Q ? dims.q_slots : dims.k_slots;
+  const int total = dims.h * nslots;
+  const int32_t* members = IS_Q ? buf.q_members : buf.k_members;
+  const int32_t* gstart = IS_Q ? buf.q_gstart : buf.k_gstart;
+  const int32_t* gcount = IS_Q ? buf.q_gcount : buf.k_gcount;
+  T* Xt = reinterpret_cast<T*>(IS_Q ? buf.q_tilde : buf.k_tilde);
+  T* Vt = reinterpret_cast<T*>(buf.v_tilde);
   float* dmean = IS_Q ? dbg.q_means : dbg.k_means;
   uint32_t elig = 0;
-
-  // 3. destination groups.  Rows are read as 16-byte chunks: lane l owns
-  //    chunk l % CPR, and the RPI row groups of a warp (CPR lanes each) work
-  //    on RPI different destination groups at once, each fetching up to kU
-  //    member rows before summing them -- up to RPI * kU rows in flight per
-  //    warp.  Members are summed in member order (destination first, then
-  //    merged sources by ascending in-block index); a member's deviation is
-  //    reduced over the CPR lanes of its row group.
-  using Ch = Chunk<T, D>;
-  constexpr int CPR = Ch::CPR, RPI = Ch::RPI, EPC = Ch::EPC, kU = 8;
-  const int rg = lane / CPR, ch = lane % CPR;
-  for (int m0 = warp * RPI; m0 < ndst; m0 += nwarps * RPI) {
-    const int m = m0 + rg;
-    const bool live = m < ndst;
-    const int c = live ? cm[m] + 1 : 0;    // members: the destination and its merged sources
+  const int step = gridDim.x * (blockDim.x >> 5) * RPI;
+  int g0 = (blockIdx.x * (blockDim.x >> 5) + (tid >> 5)) * RPI;
+  // the slot this row group handles next: count, start, first member tokens
+  auto fetch = [&](int gsl, int& c, int& gs, int (&tk)[kU]) {
+    c = 0;
+    gs = 0;
+    if (gsl < total) {
+      c = gcount[gsl];
+      gs = gstart[gsl];
+      const size_t tb = (size_t)(gsl / nslots) * dims.N;
+#pragma unroll
+      for (int u = 0; u < kU; ++u) tk[u] = u < c ? members[tb + gs + u] : 0;
+    }
+  };
+  int c, gs, tk[kU];
+  fetch(g0 + rg, c, gs, tk);
+  for (; g0 < total; g0 += step) {
+    const int gsl = g0 + rg;
+    const int hh = gsl < total ? (int)(gsl / nslots) : 0;
+    const size_t tokbase = (size_t)hh * dims.N;
+    const T* Xh = X + tokbase * D;
+    const T* Vh = IS_Q ? nullptr : V + tokbase * D;
     const int cmax = __reduce_max_sync(0xffffffffu, c);
-    const int ms = live ? gsm[m] : 0;      // first merged member in mem[]
-    const int slot = slot_off + m;
-    const int tok0 = live ? dtok[m] : 0;
-    auto member = [&](int q) -> int { return q == 0 ? tok0 : tokm[ms + q - 1]; };
     float acc[EPC], accv[EPC];
 #pragma unroll
     for (int e = 0; e < EPC; ++e) acc[e] = accv[e] = 0.f;
-    uint4 xk[kU];                  // the first kU member chunks, kept for the deviations
-    for (int q0 = 0; q0 < cmax; q0 += kU) {
+    uint4 xk[kU];
+    int tk0[kU];
+    // first batch: member indices are already here
+    {
       uint4 x[kU], xv[kU];
 #pragma unroll
       for (int u = 0; u < kU; ++u) {
-        if (q0 + u < c) {
-          const size_t off = (size_t)member(q0 + u) * D;
-          x[u] = Ch::load(Xh + off, ch);
-          if (!IS_Q) xv[u] = Ch::load(Vh + off, ch);
+        tk0[u] = tk[u];
+        if (u < c) {
+          x[u] = Ch::load(Xh + (size_t)tk[u] * D, ch);
+          if (!IS_Q) xv[u] = Ch::load(Vh + (size_t)tk[u] * D, ch);
         }
       }
+      const int c_cur = c, gs_cur = gs;
+      fetch(g0 + step + rg, c, gs, tk);         // next slot, while these rows arrive
 #pragma unroll
       for (int u = 0; u < kU; ++u) {
-        if (q0 + u < c) {
+        if (u < c_cur) {
           Ch::add(acc, x[u]);
           if (!IS_Q) Ch::add(accv, xv[u]);
         }
+        xk[u] = x[u];
       }
-      if (q0 == 0) {
+      // members beyond the first batch (large groups)
+      for (int q0 = kU; q0 < cmax; q0 += kU) {
+        int tq[kU];
 #pragma unroll
-        for (int u = 0; u < kU; ++u) xk[u] = x[u];
-      }
-    }
-    if (live) {
-      const float fc = (float)c;
+        for (int u = 0; u < kU; ++u) {
+          tq[u] = q0 + u < c_cur ? members[tokbase + gs_cur + q0 + u] : 0;
+          if (q0 + u < c_cur) {
+            x[u] = Ch::load(Xh + (size_t)tq[u] * D, ch);
+            if (!IS_Q) xv[u] = Ch::load(Vh + (size_t)tq[u] * D, ch);
+          }
+        }
 #pragma unroll
-      for (int e = 0; e < EPC; ++e) {
-        acc[e] = acc[e] / fc;
-        accv[e] = accv[e] / fc;
+        for (int u = 0; u < kU; ++u) {
+          if (q0 + u < c_cur) {
+            Ch::add(acc, x[u]);
+            if (!IS_Q) Ch::add(accv, xv[u]);
+          }
+        }
       }
-      Ch::store(Xt + (size_t)slot * D, ch, acc);
-      if (dmean) Ch::store_f32(dmean + ((size_t)hh * nslots + slot) * D, ch, acc);
-      if (!IS_Q) {
-        Ch::store(Vt + (size_t)slot * D, ch, accv);
-        if (dbg.v_means) Ch::store_f32(dbg.v_means + ((size_t)hh * nslots + slot) * D, ch, accv);
-      }
-    }
-    const int pos = live ? b.tok_off + gsm[m] + m : 0;
-    if (IS_Q && live && ch == 0) {
-      buf.q_gstart[(size_t)hh * nslots + slot] = pos;
-      buf.q_gcount[(size_t)hh * nslots + slot] = c;
-    }
-    for (int q0 = 0; q0 < cmax; q0 += kU) {
+      const bool live = gsl < total;
+      if (live) {
+        const float inv = 1.f / (float)c_cur;
 #pragma unroll
-      for (int u = 0; u < kU; ++u) {
-        const int q = q0 + u;
-        const bool mine = q < c;
-        const int tok = mine ? member(q) : 0;
-        if (IS_Q) {
-          uint4 xr = xk[u];
-          if (q0 > 0 && mine && c >= 2) xr = Ch::load(Xh + (size_t)tok * D, ch);
-          const float ss = Ch::within_row(mine ? Ch::sq_dist(xr, acc) : 0.f);
-          if (mine && ch == 0) {
-            const uint32_t key = c >= 2 ? __float_as_uint(sqrtf(ss)) + 1u : 0u;
-            buf.q_members[tokbase + pos + q] = tok;
-            buf.q_slot[tokbase + tok] = slot;
-            buf.keys[tokbase + tok] = key;
-            if (key) {
-              atomicAdd(&hist[key >> 21], 1u);
-              ++elig;
+        for (int e = 0; e < EPC; ++e) {
+          acc[e] *= inv;
+          accv[e] *= inv;
+        }
+        const size_t row = (size_t)gsl;       // = head * nslots + slot
+        Ch::store(Xt + row * D, ch, acc);
+        if (dmean) Ch::store_f32(dmean + row * D, ch, acc);
+        if (!IS_Q) {
+          Ch::store(Vt + row * D, ch, accv);
+          if (dbg.v_means) Ch::store_f32(dbg.v_means + row * D, ch, accv);
+        }
+      }
+      if (IS_Q) {
+        for (int q0 = 0; q0 < cmax; q0 += kU) {
+#pragma unroll
+          for (int u = 0; u < kU; ++u) {
+            const int q = q0 + u;
+            const bool mine = q < c_cur;
+            const int tok = q0 == 0 ? tk0[u] : (mine ? members[tokbase + gs_cur + q] : 0);
+            uint4 xr = xk[u];
+            if (q0 > 0 && mine) xr = Ch::load(Xh + (size_t)tok * D, ch);
+            const float ss = Ch::within_row(mine && c_cur >= 2 ? Ch::sq_dist(xr, acc) : 0.f);
+            if (mine && ch == 0) {
+              const uint32_t key = c_cur >= 2 ? __float_as_uint(sqrtf(ss)) + 1u : 0u;
+              buf.keys[tokbase + tok] = key;
+              if (key) {
+                atomicAdd(&hist[key >> 21], 1u);
+                ++elig;
+              }
             }
           }
-        } else if (mine && dbg.k_slot && ch == 0) {
-          dbg.k_slot[tokbase + tok] = slot;
         }
       }
     }
   }
-
-  // 4. kept sources: singleton slots after the destination groups, copied
-  //    RPI * kU rows per warp step.
-  for (int p0 = r + warp * RPI * kU; p0 < nsrc; p0 += nwarps * RPI * kU) {
-    uint4 x[kU], xv[kU];
-    int tk[kU];
-#pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      const int p = p0 + rg + RPI * u;
-      tk[u] = p < nsrc ? tokm[p] : 0;
-      if (p < nsrc) {
-        x[u] = Ch::load(Xh + (size_t)tk[u] * D, ch);
-        if (!IS_Q) xv[u] = Ch::load(Vh + (size_t)tk[u] * D, ch);
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      const int p = p0 + rg + RPI * u;
-      if (p >= nsrc) continue;
-      const int rank = p - r;
-      const int slot = slot_off + ndst + rank;
-      const int tok = tk[u];
-      Ch::store_raw(Xt + (size_t)slot * D, ch, x[u]);
-      if (dmean) Ch::store_raw_f32(dmean + ((size_t)hh * nslots + slot) * D, ch, x[u]);
-      if (!IS_Q) {
-        Ch::store_raw(Vt + (size_t)slot * D, ch, xv[u]);
-        if (dbg.v_means) Ch::store_raw_f32(dbg.v_means + ((size_t)hh * nslots + slot) * D, ch, xv[u]);
-        if (dbg.k_slot && ch == 0) dbg.k_slot[tokbase + tok] = slot;
-      } else if (ch == 0) {
-        const int pos = b.tok_off + ndst + r + rank;
-        buf.q_members[tokbase + pos] = tok;
-        buf.q_slot[tokbase + tok] = slot;
-        buf.keys[tokbase + tok] = 0u;
-        buf.q_gstart[(size_t)hh * nslots + slot] = pos;
-        buf.q_gcount[(size_t)hh * nslots + slot] = 1;
-      }
-    }
-  }
-
   if (IS_Q) {
     if (elig) atomicAdd(&s_elig, elig);
     __syncthreads();
-    for (int i = tid; i < kHistBins; i += bd)
+    for (int i = tid; i < kHistBins; i += blockDim.x)
       if (hist[i]) atomicAdd(&buf.hist[i], hist[i]);
     if (tid == 0 && s_elig) atomicAdd(&buf.state->n_eligible, s_elig);
   }
 }
 
-// Restore (key design 3): every regular query slot holding outliers becomes
-// the mean of its remaining members; a slot whose members are all outliers
-// is drained (zeros; no token reads it).
+// Restore (key design 3), flat over every (head, query slot): a slot holding
+// outliers becomes the mean of its remaining members (in member order); a
+// slot whose members are all outliers is drained (zeros; no token reads it).
 template <class T, int D>
 __global__ void __launch_bounds__(256)
-restore_kernel(Dims dims, const BlockDesc* __restrict__ blocks, const T* __restrict__ Q, Buffers buf,
-               Debug dbg) {
-  using Row = WarpRow<T, D>;
-  constexpr int E = Row::E;
+restore_kernel(Dims dims, const T* __restrict__ Q, Buffers buf, Debug dbg) {
+  using Ch = Chunk<T, D>;
+  constexpr int CPR = Ch::CPR, RPI = Ch::RPI, EPC = Ch::EPC, kU = 4;
   if (plan_failed(buf.state)) return;
   if (buf.state->sel[3] == 0 && dbg.q_restored == nullptr) return;  // no outlier anywhere
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  const int hh = blockIdx.y;
-  const BlockDesc b = blocks[blockIdx.x];
-  const size_t tokbase = (size_t)hh * dims.N;
-  const T* Qh = Q + tokbase * D;
-  T* Qt = reinterpret_cast<T*>(buf.q_tilde) + (size_t)hh * dims.q_slots * D;
-  const int nslot_b = b.n_b - b.q_r;
-  for (int s = warp; s < nslot_b; s += nwarps) {
-    const int slot = b.q_slot_off + s;
-    const int gs = buf.q_gstart[(size_t)hh * dims.q_slots + slot];
-    const int gc = buf.q_gcount[(size_t)hh * dims.q_slots + slot];
-    if (gc < 2 && dbg.q_restored == nullptr) continue;
-    if (gs < 0 || gc < 1 || gs + gc > dims.N) {
-      if (lane == 0) set_status(buf.state, HTTM_DEV_BOUNDS);
-      continue;
+  const int lane = threadIdx.x & 31;
+  const int rg = lane / CPR, ch = lane % CPR;
+  const long long total = (long long)dims.h * dims.q_slots;
+  T* Qt = reinterpret_cast<T*>(buf.q_tilde);
+  const long long nwarp_total = (long long)gridDim.x * (blockDim.x >> 5);
+  for (long long g0 = ((long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * RPI; g0 < total;
+       g0 += nwarp_total * RPI) {
+    const long long gsl = g0 + rg;
+    const bool live = gsl < total;
+    const int hh = live ? (int)(gsl / dims.q_slots) : 0;
+    const size_t tokbase = (size_t)hh * dims.N;
+    int c = live ? buf.q_gcount[gsl] : 0;
+    const int gs = live ? buf.q_gstart[gsl] : 0;
+    if (c < 0 || gs < 0 || gs + c > dims.N) {
+      if (ch == 0) set_status(buf.state, HTTM_DEV_BOUNDS);
+      c = 0;
     }
+    // outliers among the members (the lanes of the row group share them out)
     int nout = 0;
-    for (int q = lane; q < gc; q += 32) {
-      const int tok = buf.q_members[tokbase + gs + q];
-      if (tok < 0 || tok >= dims.N) {
-        set_status(buf.state, HTTM_DEV_BOUNDS);
-        continue;
+    if (c >= 2) {
+      for (int q = ch; q < c; q += CPR) {
+        const int tok = buf.q_members[tokbase + gs + q];
+        nout += (tok >= 0 && tok < dims.N) ? (buf.mask[tokbase + tok] != 0) : 0;
       }
-      nout += buf.mask[tokbase + tok] != 0;
     }
-    nout = __reduce_add_sync(0xffffffffu, nout);
-    if (nout == 0 && dbg.q_restored == nullptr) continue;
-    float acc[E], x[E];
 #pragma unroll
-    for (int e = 0; e < E; ++e) acc[e] = 0.f;
-    for (int q = 0; q < gc; ++q) {
-      const int tok = buf.q_members[tokbase + gs + q];
-      if (tok < 0 || tok >= dims.N || buf.mask[tokbase + tok]) continue;
-      Row::load(Qh + (size_t)tok * D, lane, x);
+    for (int o = 1; o < CPR; o <<= 1) nout += __shfl_xor_sync(0xffffffffu, nout, o);
+    const bool work = live && (nout > 0 || (dbg.q_restored != nullptr && c >= 1));
+    const int cw = work ? c : 0;
+    const int cmax = __reduce_max_sync(0xffffffffu, cw);
+    if (cmax == 0) continue;
+    float acc[EPC];
 #pragma unroll
-      for (int e = 0; e < E; ++e) acc[e] += x[e];
+    for (int e = 0; e < EPC; ++e) acc[e] = 0.f;
+    for (int q0 = 0; q0 < cmax; q0 += kU) {
+      uint4 x[kU];
+      bool use[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        use[u] = false;
+        if (q0 + u < cw) {
+          const int tok = buf.q_members[tokbase + gs + q0 + u];
+          use[u] = tok >= 0 && tok < dims.N && buf.mask[tokbase + tok] == 0;
+          if (use[u]) x[u] = Ch::load(Q + (tokbase + tok) * D, ch);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kU; ++u)
+        if (use[u]) Ch::add(acc, x[u]);
     }
-    const int remain = gc - nout;
+    if (!work) continue;
+    const int remain = c - nout;
 #pragma unroll
-    for (int e = 0; e < E; ++e) acc[e] = remain ? acc[e] / (float)remain : 0.f;
-    if (nout > 0) Row::store(Qt + (size_t)slot * D, lane, acc);
+    for (int e = 0; e < EPC; ++e) acc[e] = remain ? acc[e] / (float)remain : 0.f;
+    if (nout > 0) Ch::store(Qt + (size_t)gsl * D, ch, acc);
     if (dbg.q_restored) {
-      float o[E];
+      float o[EPC];
 #pragma unroll
-      for (int e = 0; e < E; ++e) o[e] = remain ? acc[e] : __int_as_float(0x7fc00000);
-      store_f32<E>(dbg.q_restored + ((size_t)hh * dims.q_slots + slot) * D, lane, D, o);
+      for (int e = 0; e < EPC; ++e) o[e] = remain ? acc[e] : __int_as_float(0x7fc00000);
+      Ch::store_f32(dbg.q_restored + (size_t)gsl * D, ch, o);
     }
   }
 }
@@ -605,29 +681,24 @@ __global__ void zero_state_kernel(Buffers buf) {
   if (threadIdx.x < 8) buf.state->sel[threadIdx.x] = 0u;
 }
 
-int next_pow2(int x) {
-  int p = 32;
-  while (p < x) p <<= 1;
-  return p;
+int gather_grid(long long units) {
+  return (int)std::max<long long>(1, std::min<long long>((units + 7) / 8, 148 * 8));
 }
 
 template <class T, int D>
-cudaError_t launch_merge_t(const Dims& dims, const BlockDesc* blocks, bool is_q, bool injected,
-                           const void* X, const void* V, const Buffers& buf, const Debug& dbg,
-                           cudaStream_t s) {
+cudaError_t launch_merge_t(const Dims& dims, const BlockDesc* blocks, bool injected, const void* Q, const void* K,
+                           const void* V, const Buffers& buf, const Debug& dbg, cudaStream_t s) {
   const int cap = (dims.max_nsrc + kMergeThreads - 1) / kMergeThreads * kMergeThreads;
-  const size_t smem = (size_t)cap * 13 + 3ull * dims.max_ndst * 4 + 2ull * kHistBins * 4 + 64 * 4;
-  dim3 grid(dims.nblk, dims.h);
-  cudaError_t e;
-  if (is_q) {
-    auto k = merge_kernel<T, D, true>;
-    if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e;
-    k<<<grid, kMergeThreads, smem, s>>>(dims, blocks, (const T*)X, nullptr, buf, dbg, injected, cap);
-  } else {
-    auto k = merge_kernel<T, D, false>;
-    if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e;
-    k<<<grid, kMergeThreads, smem, s>>>(dims, blocks, (const T*)X, (const T*)V, buf, dbg, injected, cap);
-  }
+  const size_t smem = (size_t)cap * 13 + 3ull * dims.max_ndst * 4 + (size_t)kHistBins * 4 + 64 * 4;
+  cudaError_t e = cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  plan_kernel<<<dim3(dims.nblk, dims.h, 2), kMergeThreads, smem, s>>>(dims, blocks, buf, dbg, injected ? 1 : 0, cap);
+  constexpr int RPI = Chunk<T, D>::RPI;
+  // resident warps handle several slots each, so that prefetching pays
+  gather_kernel<T, D, true><<<gather_grid((long long)dims.h * dims.q_slots / (4 * RPI) + 1), 256, 0, s>>>(
+      dims, (const T*)Q, nullptr, buf, dbg);
+  gather_kernel<T, D, false><<<gather_grid((long long)dims.h * dims.k_slots / (4 * RPI) + 1), 256, 0, s>>>(
+      dims, (const T*)K, (const T*)V, buf, dbg);
   return cudaGetLastError();
 }
 
@@ -638,26 +709,31 @@ cudaError_t launch_zero_state(const Dims&, const Buffers& buf, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_merge(const Dims& dims, bool fp32, const BlockDesc* blocks, bool is_q, bool injected,
-                         const void* X, const void* V, const Buffers& buf, const Debug& dbg,
-                         cudaStream_t s) {
+cudaError_t launch_merge(const Dims& dims, bool fp32, const BlockDesc* blocks, bool injected, const void* Q,
+                         const void* K, const void* V, const Buffers& buf, const Debug& dbg, cudaStream_t s) {
   if (fp32) {
-    if (dims.d == 16) return launch_merge_t<float, 16>(dims, blocks, is_q, injected, X, V, buf, dbg, s);
-    return launch_merge_t<float, 64>(dims, blocks, is_q, injected, X, V, buf, dbg, s);
+    if (dims.d == 16) return launch_merge_t<float, 16>(dims, blocks, injected, Q, K, V, buf, dbg, s);
+    return launch_merge_t<float, 64>(dims, blocks, injected, Q, K, V, buf, dbg, s);
   }
-  if (dims.d == 16) return launch_merge_t<__nv_bfloat16, 16>(dims, blocks, is_q, injected, X, V, buf, dbg, s);
-  return launch_merge_t<__nv_bfloat16, 64>(dims, blocks, is_q, injected, X, V, buf, dbg, s);
+  if (dims.d == 16) return launch_merge_t<__nv_bfloat16, 16>(dims, blocks, injected, Q, K, V, buf, dbg, s);
+  return launch_merge_t<__nv_bfloat16, 64>(dims, blocks, injected, Q, K, V, buf, dbg, s);
 }
 
-cudaError_t launch_restore(const Dims& dims, bool fp32, const BlockDesc* blocks, const void* Q,
-                           const Buffers& buf, const Debug& dbg, cudaStream_t s) {
-  dim3 grid(dims.nblk, dims.h);
+cudaError_t launch_restore(const Dims& dims, bool fp32, const BlockDesc*, const void* Q, const Buffers& buf,
+                           const Debug& dbg, cudaStream_t s) {
+  const long long units = (long long)dims.h * dims.q_slots;
   if (fp32) {
-    if (dims.d == 16) restore_kernel<float, 16><<<grid, 256, 0, s>>>(dims, blocks, (const float*)Q, buf, dbg);
-    else restore_kernel<float, 64><<<grid, 256, 0, s>>>(dims, blocks, (const float*)Q, buf, dbg);
+    if (dims.d == 16)
+      restore_kernel<float, 16><<<gather_grid(units / Chunk<float, 16>::RPI + 1), 256, 0, s>>>(dims, (const float*)Q, buf, dbg);
+    else
+      restore_kernel<float, 64><<<gather_grid(units / Chunk<float, 64>::RPI + 1), 256, 0, s>>>(dims, (const float*)Q, buf, dbg);
   } else {
-    if (dims.d == 16) restore_kernel<__nv_bfloat16, 16><<<grid, 256, 0, s>>>(dims, blocks, (const __nv_bfloat16*)Q, buf, dbg);
-    else restore_kernel<__nv_bfloat16, 64><<<grid, 256, 0, s>>>(dims, blocks, (const __nv_bfloat16*)Q, buf, dbg);
+    if (dims.d == 16)
+      restore_kernel<__nv_bfloat16, 16><<<gather_grid(units / Chunk<__nv_bfloat16, 16>::RPI + 1), 256, 0, s>>>(
+          dims, (const __nv_bfloat16*)Q, buf, dbg);
+    else
+      restore_kernel<__nv_bfloat16, 64><<<gather_grid(units / Chunk<__nv_bfloat16, 64>::RPI + 1), 256, 0, s>>>(
+          dims, (const __nv_bfloat16*)Q, buf, dbg);
   }
   return cudaGetLastError();
 }
