@@ -37,6 +37,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true", help="skip the 500-frame layer")
     return ap.parse_args()
 
 
@@ -164,17 +165,138 @@ class Clocks:
 # our arm
 # ----------------------------------------------------------------------------
 
-def traffic_record(kernel_file: str):
-    """DRAM bytes per launch from a committed ncu summary, if the kernel source
-    is unchanged since it was captured (else None)."""
+def traffic_record(kernel_file: str, workload: str):
+    """DRAM bytes per launch of a kernel on a workload, from a committed ncu
+    summary (profiles/traffic.json), if the kernel source is unchanged since
+    the counters were taken (else None)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
-    rec = json.load(open(p)).get(os.path.basename(kernel_file))
+    rec = json.load(open(p)).get(os.path.basename(kernel_file), {}).get(workload)
     if not rec:
         return None
     sha = hashlib.sha256(open(kernel_file, "rb").read()).hexdigest()[:16]
     return rec if rec.get("source_sha") == sha else None
+
+
+def max_over_ranks(value: float, world: int, device) -> float:
+    """The largest of every rank's value (each rank times its own layer; the
+    job's step time is the slowest rank's)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def measure_layer(w, steps: int, warmup: int, rank: int, world: int, dev, with_e2e: bool = True):
+    """Time `steps` forward calls of one layer (inputs resident in HBM) with
+    stage events on, then the same call end to end from pinned host memory."""
+    import torch
+    import torch.distributed as dist
+
+    from token_merging_view_b200 import binding as B
+    from token_merging_view_b200.inputs import make_qkv
+
+    Q, K, V = make_qkv(T=w.T, grid=w.grid, h=w.h, d=w.d, seed=w.seed + 1000 * rank, noise_sigma=w.noise_sigma,
+                       max_shift=w.max_shift, dtype=torch.float32 if w.fp32 else torch.bfloat16, device=dev)
+    plan = B.httm_plan(B.LayerConfig.from_workload(w))
+    ws = plan.new_workspace(dev)
+    out = torch.empty_like(Q)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        B.httm_forward(plan, Q, K, V, out=out, workspace=ws, stream=stream)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    assert B.httm_get_device_status(plan, ws) == 0
+    n_out = B.workspace_view(plan, ws, "n_out").cpu()
+    sum_lq = w.h * plan.info.q_slots + int(n_out.sum())
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def timed(fn, n):
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n):
+            fn()
+        b.record(stream)
+        barrier()
+        return max_over_ranks(a.elapsed_time(b), world, dev)
+
+    clocks = Clocks(dev.index if dev.index is not None else 0)
+    plan.profile(True)
+    plan.profile_read()
+    total_ms = timed(step, steps)
+    stages = plan.profile_read()
+    plan.profile(False)
+    clk = clocks.stop()
+    res = {"plan": plan, "Q": Q, "K": K, "V": V, "ms_step": total_ms / steps, "stages": stages, "sum_lq": sum_lq,
+           "launches": plan.launches() * steps, "clocks": clk}
+    if with_e2e:
+        # end to end through the same C ABI call: pinned host Q/K/V in, host out back
+        hQ, hK, hV = (t.cpu().pin_memory() for t in (Q, K, V))
+        hO = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+
+        def e2e_step():
+            Q.copy_(hQ, non_blocking=True)
+            K.copy_(hK, non_blocking=True)
+            V.copy_(hV, non_blocking=True)
+            step()
+            hO.copy_(out, non_blocking=True)
+
+        e2e_step()
+        n = max(2, steps // 2)
+        res["e2e_ms"] = timed(e2e_step, n) / n
+        res["h2d"] = 3 * Q.numel() * Q.element_size()
+        res["d2h"] = out.numel() * out.element_size()
+    return res
+
+
+def roofline_of(w, r, steps: int):
+    """Attention (the dominant kernel) against the bf16 tensor peak, and the
+    memory-bound stages against the HBM copy bandwidth."""
+    import token_merging_view_b200 as pkg
+    pk, pk_kind = peaks()
+    plan = r["plan"]
+    att_ms, att_n = r["stages"]["attention"]
+    att_avg_ms = att_ms / max(1, att_n)
+    flops = 4.0 * w.d * plan.info.kv_slots * r["sum_lq"]
+    achieved = flops / (att_avg_ms / 1e3) / 1e12
+    peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+    att_src = os.path.join(os.path.dirname(pkg.__file__), "csrc", "attn_tc.cu")
+    tr = traffic_record(att_src, w.name)
+    roof = {"bound": "tensor", "kernel": "attention (attn_tc_kernel)", "achieved": round(achieved, 2),
+            "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+            "peak_kind": f"{pk_kind} bf16 sustained (kernel timed inside a long step); burst {pk['bf16_tflops']}",
+            "frac_of_burst": round(achieved / pk["bf16_tflops"], 4),
+            "traffic": tr["bytes_per_launch"] if tr else None,
+            "algorithmic_flops_per_launch": flops, "avg_launch_ms": round(att_avg_ms, 4)}
+    es = 4 if w.fp32 else 2
+    row = w.d * es
+    hn = w.h * w.N
+    mem_bytes = {
+        # read Q, K, V; write Q~ (regular slots), K~, V~; per-token slot and deviation key
+        "merge": 3 * hn * row + (w.h * plan.info.q_slots + 2 * w.h * plan.info.kv_slots) * row + 8 * hn,
+        # read O~ once, write out in original order, read the slot map
+        "unmerge": hn * row + r["sum_lq"] * row + 4 * hn,
+    }
+    hbm = pk["hbm_gbs"]
+    mem = {}
+    for k, b in mem_bytes.items():
+        ms = r["stages"][k][0] / steps
+        if ms > 0:
+            mem[k] = {"algorithmic_bytes": b, "ms": round(ms, 4), "GBps": round(b / ms / 1e6, 1),
+                      "frac_of_measured_hbm": round(b / ms / 1e6 / hbm, 4)}
+    return roof, mem
 
 
 def run_ours(args):
@@ -191,145 +313,79 @@ def run_ours(args):
     if world > 1:
         dist.init_process_group("nccl", device_id=dev)
     w = WORKLOADS[args.workload]
-    Q, K, V = make_qkv(T=w.T, grid=w.grid, h=w.h, d=w.d, seed=w.seed + 1000 * rank, noise_sigma=w.noise_sigma,
-                       max_shift=w.max_shift, dtype=torch.float32 if w.fp32 else torch.bfloat16, device=dev)
-    plan = B.httm_plan(B.LayerConfig.from_workload(w))
-    ws = plan.new_workspace(dev)
-    out = torch.empty_like(Q)
-    stream = torch.cuda.current_stream()
-
-    def step():
-        B.httm_forward(plan, Q, K, V, out=out, workspace=ws, stream=stream)
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    assert B.httm_get_device_status(plan, ws) == 0
-    n_out = B.workspace_view(plan, ws, "n_out").cpu()
-    sum_lq = w.h * plan.info.q_slots + int(n_out.sum())
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize()
-
-    def timed(fn, steps):
-        barrier()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(steps):
-            fn()
-        b.record(stream)
-        barrier()
-        ms = a.elapsed_time(b)
-        if world > 1:
-            t = torch.tensor([ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms = float(t.item())
-        return ms
-
-    clocks = Clocks(local)
-    plan.profile(True)
-    plan.profile_read()
-    total_ms = timed(step, args.steps)
-    stages = plan.profile_read()
-    plan.profile(False)
-    clk = clocks.stop()
-    launches = plan.launches() * args.steps
-    ms_step = total_ms / args.steps
+    r = measure_layer(w, args.steps, args.warmup, rank, world, dev)
+    ms_step = r["ms_step"]
     value = world * w.N / (ms_step / 1e3)
-
-    # end to end through the same C ABI call: pinned host Q/K/V in, host out back
-    hQ, hK, hV = (t.cpu().pin_memory() for t in (Q, K, V))
-    hO = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-
-    def e2e_step():
-        Q.copy_(hQ, non_blocking=True)
-        K.copy_(hK, non_blocking=True)
-        V.copy_(hV, non_blocking=True)
-        step()
-        hO.copy_(out, non_blocking=True)
-
-    e2e_step()
-    e2e_steps = max(2, args.steps // 2)
-    e2e_ms = timed(e2e_step, e2e_steps) / e2e_steps
-    h2d = 3 * Q.numel() * Q.element_size()
-    d2h = out.numel() * out.element_size()
-
-    # the dominant kernel: attention on the shortened sequences
-    pk, pk_kind = peaks()
-    att_ms, att_n = stages["attention"]
-    att_avg_ms = att_ms / max(1, att_n)
-    flops = 4.0 * w.d * plan.info.kv_slots * sum_lq
-    achieved = flops / (att_avg_ms / 1e3) / 1e12
-    peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
-    import token_merging_view_b200 as pkg
-    att_src = os.path.join(os.path.dirname(pkg.__file__), "csrc", "attn_tc.cu")
-    tr = traffic_record(att_src)
-    roofline = {"bound": "tensor", "kernel": "attention", "achieved": round(achieved, 2), "peak": peak,
-                "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                "peak_kind": f"{pk_kind} bf16 sustained (kernel timed inside a long step)",
-                "traffic": tr["bytes_per_launch"] if tr else None,
-                "algorithmic_flops_per_launch": flops, "avg_launch_ms": round(att_avg_ms, 4)}
-
-    # memory-bound stages against HBM
+    roof, mem = roofline_of(w, r, args.steps)
+    Q = r["Q"]
     es = 4 if w.fp32 else 2
-    row = w.d * es
-    mem_bytes = {
-        "merge": (3 * w.h * w.N * row + (w.h * plan.info.q_slots + 2 * w.h * plan.info.kv_slots) * row),
-        "unmerge": (w.h * w.N * row + sum_lq * row + w.h * w.N * 4),
-    }
-    hbm = pk["hbm_gbs"]
-    per_step = {k: round(v[0] / args.steps, 4) for k, v in stages.items()}
-    mem_roof = {}
-    for k, b in mem_bytes.items():
-        ms = stages[k][0] / args.steps
-        if ms > 0:
-            mem_roof[k] = {"algorithmic_bytes": b, "ms": round(ms, 4), "GBps": round(b / ms / 1e6, 1),
-                           "frac_of_measured_hbm": round(b / ms / 1e6 / hbm, 4)}
 
     dense = None
     if not args.no_dense and rank == 0 and world == 1:
         dplan = B.httm_plan(B.LayerConfig.from_workload(w, mode=B.HTTM_DENSE))
         dws = dplan.new_workspace(dev)
-        B.httm_forward(dplan, Q, K, V, out=out, workspace=dws)
+        out = torch.empty_like(Q)
+        Kd, Vd = r["K"], r["V"]
+        B.httm_forward(dplan, Q, Kd, Vd, out=out, workspace=dws)
         torch.cuda.synchronize()
+        stream = torch.cuda.current_stream()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        B.httm_forward(dplan, Q, K, V, out=out, workspace=dws, stream=stream)
+        B.httm_forward(dplan, Q, Kd, Vd, out=out, workspace=dws, stream=stream)
         b.record(stream)
         torch.cuda.synchronize()
         dms = a.elapsed_time(b)
         dflops = 4.0 * w.d * w.h * float(w.N) * w.N
         dense = {"tokens_per_s": round(w.N / (dms / 1e3), 1), "ms": round(dms, 3),
                  "TFLOPs": round(dflops / (dms / 1e3) / 1e12, 2)}
-        del dws, dplan
+        del dws, dplan, out, Kd, Vd
+    plan_info = (r["plan"].info.q_slots, r["plan"].info.kv_slots)
+    sum_lq = r["sum_lq"]
+    e2e = {"value": round(world * w.N / (r["e2e_ms"] / 1e3), 1), "unit": "tokens/s",
+           "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]}
+    launches, clk, stages = r["launches"], r["clocks"], r["stages"]
+    del r, Q
+    torch.cuda.empty_cache()
+
+    secondary = None
+    if not args.no_secondary and world == 1 and args.workload != "vggt_500f":
+        w2 = WORKLOADS["vggt_500f"]
+        r2 = measure_layer(w2, 3, 2, rank, world, dev, with_e2e=False)
+        roof2, mem2 = roofline_of(w2, r2, 3)
+        secondary = {"workload": w2.name, "tokens": w2.N, "value": round(w2.N / (r2["ms_step"] / 1e3), 1),
+                     "unit": "tokens/s", "ms_per_step": round(r2["ms_step"], 3), "steps": 3,
+                     "roofline": roof2, "memory_stages": mem2,
+                     "stage_ms_per_step": {k: round(v[0] / 3, 4) for k, v in r2["stages"].items()}}
+        del r2
+        torch.cuda.empty_cache()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rows = 512 if w.N <= 200_000 else 128
-        cpu = oracle_sample(w, Q, K, V, rows)
+        Qc, Kc, Vc = make_qkv(T=w.T, grid=w.grid, h=1, d=w.d, seed=w.seed, noise_sigma=w.noise_sigma,
+                              max_shift=w.max_shift, dtype=torch.float32 if w.fp32 else torch.bfloat16)
+        cpu = oracle_sample(w, Qc, Kc, Vc, 512 if w.N <= 200_000 else 128)
         cpu.pop("measured_s", None)
 
     if rank == 0:
         line = {
             "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if not w.fp32 else "f32",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32" if w.fp32 else "bf16",
             "data": "synthetic (seeded blurred-field Q/K/V, VGGT global-attention shapes)",
             "config": {"workload": w.name, "frames": w.T, "patches_per_frame": w.P, "tokens": w.N, "heads": w.h,
                        "d_head": w.d, "n_s": w.n_s, "n_t": w.n_t, "q_dst_stride": w.q_stride,
                        "kv_dst_stride": w.kv_stride, "q_merge_pct": w.q_pct, "kv_merge_pct": w.kv_pct,
-                       "outlier_pct": w.out_pct, "q_rows": sum_lq, "kv_rows_per_head": plan.info.kv_slots,
-                       "parallelism": f"replicas x{world}" if world > 1 else "single",
-                       "l2": f"inputs larger than L2 ({3 * Q.numel() * es / 2**20:.0f} MiB of Q/K/V vs 126 MB)"},
-            "e2e": {"value": round(world * w.N / (e2e_ms / 1e3), 1), "unit": "tokens/s",
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                       "outlier_pct": w.out_pct, "q_rows": sum_lq, "kv_rows_per_head": plan_info[1],
+                       "parallelism": f"independent layer per GPU x{world}" if world > 1 else "single GPU",
+                       "l2": f"inputs larger than L2 ({3 * w.h * w.N * w.d * es / 2**20:.0f} MiB of Q/K/V vs 126 MB)"},
+            "e2e": e2e,
             "gpu_launches": launches,
-            "roofline": roofline,
-            "memory_stages": mem_roof,
-            "stage_ms_per_step": per_step,
+            "roofline": roof,
+            "memory_stages": mem,
+            "stage_ms_per_step": {k: round(v[0] / args.steps, 4) for k, v in stages.items()},
             "dense_attention_same_length": dense,
+            "secondary_workload": secondary,
             "clocks": clk,
             "cpu_baseline": cpu,
         }

@@ -103,6 +103,13 @@ def test_vggt_100f_layer_sampled():
     _full_check(WORKLOADS["vggt_100f"], tokens_per_head=128)
 
 
+@pytest.mark.slow
+def test_vggt_500f_layer_sampled():
+    """The 500-frame layer (684,500 tokens, queries with destinations every
+    8th token and 85% merged) in the launch configuration bench.py times."""
+    _full_check(WORKLOADS["vggt_500f"], tokens_per_head=48)
+
+
 def test_reorder_matches_oracle():
     for w in (TINY, MID, MID.with_(mode=CONTIGUOUS, contig_block=500)):
         _, plan, cfg, (Q, _, _), (q, _, _) = _case(w)

@@ -529,14 +529,13 @@ restore_kernel(Dims dims, const T* __restrict__ Q, Buffers buf, Debug dbg) {
   if (buf.state->sel[3] == 0 && dbg.q_restored == nullptr) return;  // no outlier anywhere
   const int lane = threadIdx.x & 31;
   const int rg = lane / CPR, ch = lane % CPR;
-  const long long total = (long long)dims.h * dims.q_slots;
+  const int total = dims.h * dims.q_slots;          // h * N < 2^31 (plan limit)
   T* Qt = reinterpret_cast<T*>(buf.q_tilde);
-  const long long nwarp_total = (long long)gridDim.x * (blockDim.x >> 5);
-  for (long long g0 = ((long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * RPI; g0 < total;
-       g0 += nwarp_total * RPI) {
-    const long long gsl = g0 + rg;
+  const int nwarp_total = gridDim.x * (blockDim.x >> 5);
+  for (int g0 = (blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * RPI; g0 < total; g0 += nwarp_total * RPI) {
+    const int gsl = g0 + rg;
     const bool live = gsl < total;
-    const int hh = live ? (int)(gsl / dims.q_slots) : 0;
+    const int hh = live ? gsl / dims.q_slots : 0;
     const size_t tokbase = (size_t)hh * dims.N;
     int c = live ? buf.q_gcount[gsl] : 0;
     const int gs = live ? buf.q_gstart[gsl] : 0;
