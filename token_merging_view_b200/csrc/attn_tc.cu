@@ -211,19 +211,49 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         for (int i = 0; i < kBN; ++i)
           if (i >= valid) sr[i] = __float_as_uint(-INFINITY);
       }
-      // row max: four chains of three-input max
-      float mx[4];
+      // p = 2^(s * c - m) with the running max m as it stands: the affine
+      // part and the row sums on packed fp32 pairs, the exponentials on the
+      // exp unit, and the tile max tracked alongside (three-input max).  If a
+      // row's tile max exceeds m by more than 8 (log2 units) -- always on
+      // the first tile, rarely afterwards -- the warp rescales O and the sum
+      // and redoes the tile with the new max.
+      const unsigned long long cc = f2_pack(scale_log2, scale_log2);
+      float rsum = 0.f;
+      for (int pass = 0; pass < 2; ++pass) {
+        const unsigned long long mm = f2_pack(-m_used, -m_used);
+        unsigned long long rs[4];
+        float mx[4];
 #pragma unroll
-      for (int a = 0; a < 4; ++a) mx[a] = __uint_as_float(sr[a]);
+        for (int a = 0; a < 4; ++a) {
+          rs[a] = 0ull;                                  // (0.f, 0.f)
+          mx[a] = -INFINITY;
+        }
 #pragma unroll
-      for (int i = 4; i < kBN; i += 8) {
+        for (int c = 0; c < 2; ++c) {
+          uint32_t pk[32];
 #pragma unroll
-        for (int a = 0; a < 4; ++a) mx[a] = max3(mx[a], __uint_as_float(sr[i + a]), __uint_as_float(sr[i + 4 + a]));
-      }
-      const float mt = max3(mx[0], mx[1], fmaxf(mx[2], mx[3]));
-      const float mts = mt * scale_log2;
-      const bool need = mts > m_used + 8.f;
-      if (__any_sync(0xffffffffu, need)) {
+          for (int i = 0; i < 32; ++i) {
+            const float s0 = __uint_as_float(sr[c * 64 + 2 * i]), s1 = __uint_as_float(sr[c * 64 + 2 * i + 1]);
+            mx[i & 3] = max3(mx[i & 3], s0, s1);
+            const unsigned long long xp = f2_fma(f2_pack(s0, s1), cc, mm);
+            float x0, x1;
+            f2_unpack(xp, x0, x1);
+            const float p0 = ex2(x0), p1 = ex2(x1);
+            rs[i & 3] = f2_add(rs[i & 3], f2_pack(p0, p1));
+            pk[i] = pack_bf16(p0, p1);
+          }
+          tmem_st32(ts + c * 32, pk);
+        }
+        float r0, r1, r2, r3, r4, r5, r6, r7;
+        f2_unpack(rs[0], r0, r1);
+        f2_unpack(rs[1], r2, r3);
+        f2_unpack(rs[2], r4, r5);
+        f2_unpack(rs[3], r6, r7);
+        rsum = ((r0 + r1) + (r2 + r3)) + ((r4 + r5) + (r6 + r7));
+        if (pass == 1) break;
+        const float mts = max3(mx[0], mx[1], fmaxf(mx[2], mx[3])) * scale_log2;
+        const bool need = mts > m_used + 8.f;
+        if (!__any_sync(0xffffffffu, need)) break;
         const float m_new = fmaxf(m_used, mts);
         const float alpha = ex2(m_used - m_new);
         if (j > 0) {
@@ -245,34 +275,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         l *= alpha;
         m_used = m_new;
       }
-      // p = 2^(s * c - m): the affine part and the row sums on packed fp32
-      // pairs, the exponentials on the exp unit
-      const unsigned long long cc = f2_pack(scale_log2, scale_log2);
-      const unsigned long long mm = f2_pack(-m_used, -m_used);
-      unsigned long long rs[4];
-#pragma unroll
-      for (int a = 0; a < 4; ++a) rs[a] = 0ull;           // (0.f, 0.f)
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const unsigned long long xp =
-              f2_fma(f2_pack(__uint_as_float(sr[c * 64 + 2 * i]), __uint_as_float(sr[c * 64 + 2 * i + 1])), cc, mm);
-          float x0, x1;
-          f2_unpack(xp, x0, x1);
-          const float p0 = ex2(x0), p1 = ex2(x1);
-          rs[i & 3] = f2_add(rs[i & 3], f2_pack(p0, p1));
-          pk[i] = pack_bf16(p0, p1);
-        }
-        tmem_st32(ts + c * 32, pk);
-      }
-      float r0, r1, r2, r3, r4, r5, r6, r7;
-      f2_unpack(rs[0], r0, r1);
-      f2_unpack(rs[1], r2, r3);
-      f2_unpack(rs[2], r4, r5);
-      f2_unpack(rs[3], r6, r7);
-      l += ((r0 + r1) + (r2 + r3)) + ((r4 + r5) + (r6 + r7));
+      if (!ok) break;
+      l += rsum;
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&sm.p_full[t]);
