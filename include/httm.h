@@ -196,6 +196,27 @@ httm_status httm_forward_with_plan(httm_plan_t plan, const void* Q, const void* 
                                    void* stream);
 
 /*
+ * httm_forward_reuse: the layer on new Q, K, V with the merge indices of an
+ * earlier call kept.  The LiteVGGT note (key design 3, cross-layer cached
+ * merging) computes the merge indices once every few layers and lets the
+ * layers in between reuse them, since token similarity changes little from
+ * one layer to the next.  Here the reused state is both plans' member lists
+ * (which sources merged into which destination, per head and block) left in
+ * `workspace` by the last httm_forward / httm_forward_debug /
+ * httm_forward_with_plan call on the same plan and workspace; matching and
+ * top-r selection are skipped.  Group means of Q, K and V, the query
+ * deviations, the outlier filter and restore, attention and unmerge are all
+ * recomputed from the new inputs.  The call is otherwise httm_forward's
+ * (same arguments, asynchronous on `stream`).
+ * Errors: HTTM_ERR_ARG in HTTM_DENSE mode.  If the workspace does not hold
+ * member lists written by this plan (no earlier call, another plan's call
+ * since, or a call whose planning failed), the device sets HTTM_DEV_BAD_PLAN
+ * and the output is undefined; httm_get_device_status() reports it.
+ */
+httm_status httm_forward_reuse(httm_plan_t plan, const void* Q, const void* K, const void* V,
+                               void* out, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * httm_reorder: temporal reordering (key design 2).  inverse = 0: X in
  * original order [h, N, d] -> Xb in block order (block after block, each
  * block frame-major: the n_s-patch region of frame t0, then of t0 + 1, ...).

@@ -159,6 +159,19 @@ def test_deterministic():
         assert np.array_equal(da[key], db[key], equal_nan=True), key
 
 
+def test_output_independent_of_workspace_contents():
+    """Rows of Q~ past a work item's end are never written; attention must
+    not let them change the live rows (filled with zeros, then with large
+    finite values)."""
+    _, plan, _, (Q, K, V), _ = _case(MID)
+    outs = []
+    for fill in (0x00, 0x47):
+        ws = torch.full((plan.workspace_bytes,), fill, dtype=torch.uint8, device="cuda")
+        outs.append(B.httm_forward(plan, Q, K, V, workspace=ws))
+        assert B.httm_get_device_status(plan, ws) == 0
+    assert torch.equal(outs[0], outs[1])
+
+
 def test_invalid_injected_plan_sets_status():
     w, plan, cfg, (Q, K, V), (q, k, v) = _case(MID.with_(T=3, h=2))
     res = O.forward_plan(cfg, q, k, v)

@@ -14,6 +14,7 @@ from .binding import (  # noqa: F401
     debug_buffers,
     httm_forward,
     httm_forward_debug,
+    httm_forward_reuse,
     httm_forward_with_plan,
     httm_get_device_status,
     httm_plan,

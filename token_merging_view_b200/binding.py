@@ -24,7 +24,7 @@ HTTM_DEV_BAD_PLAN, HTTM_DEV_BOUNDS, HTTM_DEV_TIMEOUT = 0x1, 0x2, 0x4
 # every symbol include/httm.h declares
 EXPORTS = (
     "httm_plan", "httm_plan_destroy", "httm_get_plan_info", "httm_workspace_bytes",
-    "httm_forward", "httm_forward_debug", "httm_forward_with_plan", "httm_reorder",
+    "httm_forward", "httm_forward_debug", "httm_forward_with_plan", "httm_forward_reuse", "httm_reorder",
     "httm_get_device_status", "httm_forward_launches", "httm_profile_enable", "httm_profile_read",
     "httm_select_outliers_noalloc", "httm_status_str",
 )
@@ -82,6 +82,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.httm_forward_debug.argtypes = [P, V, V, V, V, V, S, ctypes.POINTER(httm_debug), V]
     lib.httm_forward_with_plan.argtypes = [P, V, V, V, V, V, S, ctypes.POINTER(httm_merge_plan),
                                            ctypes.POINTER(httm_debug), V]
+    lib.httm_forward_reuse.argtypes = [P, V, V, V, V, V, S, V]
     lib.httm_reorder.argtypes = [P, V, V, I, V]
     lib.httm_get_device_status.argtypes = [P, V, V, ctypes.POINTER(U)]
     lib.httm_forward_launches.argtypes = [P]
@@ -93,7 +94,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.httm_status_str.argtypes = [I]
     lib.httm_status_str.restype = ctypes.c_char_p
     for name in ("httm_plan", "httm_get_plan_info", "httm_forward", "httm_forward_debug",
-                 "httm_forward_with_plan", "httm_reorder", "httm_get_device_status",
+                 "httm_forward_with_plan", "httm_forward_reuse", "httm_reorder", "httm_get_device_status",
                  "httm_profile_enable", "httm_profile_read"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
@@ -263,6 +264,20 @@ def httm_forward_with_plan(plan: Plan, Q, K, V, injected: dict, dbg: dict | None
                                                  _ptr(workspace), workspace.numel(), ctypes.byref(mp),
                                                  ctypes.byref(d) if dbg else None, _stream(stream)),
            "httm_forward_with_plan")
+    return out
+
+
+def httm_forward_reuse(plan: Plan, Q, K, V, out=None, workspace=None, stream=None):
+    """The layer on new Q/K/V with the merge indices (both plans' member lists)
+    that the last full forward on ``plan`` left in ``workspace``; matching and
+    top-r selection are skipped (cached merge indices, LiteVGGT note, key
+    design 3).  ``workspace`` must be the one that forward used."""
+    if workspace is None:
+        raise ValueError("httm_forward_reuse needs the workspace of an earlier forward")
+    out, workspace = _prep(plan, Q, K, V, out, workspace)
+    _check(load_library().httm_forward_reuse(plan.handle, _ptr(Q), _ptr(K), _ptr(V), _ptr(out),
+                                             _ptr(workspace), workspace.numel(), _stream(stream)),
+           "httm_forward_reuse")
     return out
 
 

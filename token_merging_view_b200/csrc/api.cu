@@ -2,6 +2,7 @@
 // of the HTTM note: blocks of n_s patches x n_t frames), the workspace layout
 // and the launch sequence of one merged global-attention layer.
 #include <algorithm>
+#include <atomic>
 #include <cstdio>
 #include <cstring>
 #include <new>
@@ -105,6 +106,7 @@ Workspace layout(const Dims& d, bool fp32) {
   w.k_score = take((size_t)d.h * d.k_src * 4);
   w.k_merged = take((size_t)d.h * d.k_src);
   w.q_slot = take(hN * 4);
+  w.q_orank = take(hN * 4);
   w.keys = take(hN * 4);
   w.mask = take(hN);
   w.q_members = take(hN * 4);
@@ -137,6 +139,7 @@ Buffers resolve(const Workspace& w, void* base) {
   b.k_score = reinterpret_cast<float*>(p + w.k_score);
   b.k_merged = reinterpret_cast<uint8_t*>(p + w.k_merged);
   b.q_slot = reinterpret_cast<int32_t*>(p + w.q_slot);
+  b.q_orank = reinterpret_cast<int32_t*>(p + w.q_orank);
   b.keys = reinterpret_cast<uint32_t*>(p + w.keys);
   b.mask = reinterpret_cast<uint8_t*>(p + w.mask);
   b.q_members = reinterpret_cast<int32_t*>(p + w.q_members);
@@ -205,10 +208,12 @@ httm_status attention(const httm_plan_s* plan, const void* q, const void* k, con
 }
 
 httm_status forward_impl(httm_plan_s* plan, const void* Q, const void* K, const void* V, void* out, void* ws,
-                         size_t ws_bytes, const httm_merge_plan* inj, const httm_debug* dbg, void* stream) {
+                         size_t ws_bytes, const httm_merge_plan* inj, const httm_debug* dbg, void* stream,
+                         bool reuse = false) {
   if (!plan || !Q || !K || !V || !out || !ws) return HTTM_ERR_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(out)) return HTTM_ERR_ALIGN;
   if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return HTTM_ERR_ALIGN;
+  if (reuse && (inj || plan->dims.mode == HTTM_DENSE)) return HTTM_ERR_ARG;
   if (ws_bytes < plan->ws.total) return HTTM_ERR_WORKSPACE;
   if (inj) {
     const bool any = inj->q_best || inj->q_merged || inj->k_best || inj->k_merged;
@@ -231,7 +236,7 @@ httm_status forward_impl(httm_plan_s* plan, const void* Q, const void* K, const 
   int launches = 0;
   {
     StageTimer t(plan, s, HTTM_STAGE_OTHER, dims.mode == HTTM_DENSE ? 2 : 1);
-    HTTM_LAUNCH(launch_zero_state(dims, buf, s));
+    HTTM_LAUNCH(launch_zero_state(dims, buf, reuse, s));
     if (dims.mode == HTTM_DENSE) HTTM_LAUNCH(launch_dense_items(dims, buf, s));
   }
   if (dims.mode == HTTM_DENSE) {
@@ -248,7 +253,7 @@ httm_status forward_impl(httm_plan_s* plan, const void* Q, const void* K, const 
     Inject ii{inj->q_best, inj->q_merged, inj->k_best, inj->k_merged, inj->outlier};
     HTTM_LAUNCH(launch_import_plan(dims, plan->blocks_d, ii, buf, s));
   }
-  if (!plan_inj) {
+  if (!plan_inj && !reuse) {
     StageTimer t(plan, s, HTTM_STAGE_MATCH, 1);
     cudaError_t e = cudaErrorNotSupported;
     if (match_tc_supported(dims, fp32))
@@ -259,9 +264,9 @@ httm_status forward_impl(httm_plan_s* plan, const void* Q, const void* K, const 
     if (e != cudaSuccess) return HTTM_ERR_CUDA;
   }
   {
-    StageTimer t(plan, s, HTTM_STAGE_MERGE, 3);
-    HTTM_LAUNCH(launch_merge(dims, fp32, plan->blocks_d, plan_inj, Q, K, V, buf, dd, s));
-    launches += 2;  // planning, then the two gathers
+    StageTimer t(plan, s, HTTM_STAGE_MERGE, reuse ? 2 : 3);
+    HTTM_LAUNCH(launch_merge(dims, fp32, plan->blocks_d, plan_inj, reuse, Q, K, V, buf, dd, s));
+    launches += reuse ? 1 : 2;  // planning (unless reused), then the two gathers
   }
   {
     StageTimer t(plan, s, HTTM_STAGE_OUTLIER, mask_inj ? 4 : 6);
@@ -325,6 +330,7 @@ httm_status httm_plan(const httm_cfg* cfg, httm_plan_t* out) {
   }
   httm_plan_s* p = new (std::nothrow) httm_plan_s();
   if (!p) return HTTM_ERR_ARG;
+  static std::atomic<uint32_t> next_id{1};
   p->cfg = c;
   p->fp32 = c.dtype == HTTM_F32;
   Dims& d = p->dims;
@@ -340,6 +346,8 @@ httm_status httm_plan(const httm_cfg* cfg, httm_plan_t* out) {
   d.q_stride = c.q_dst_stride;
   d.kv_stride = c.kv_dst_stride;
   d.scale = c.softmax_scale > 0.f ? c.softmax_scale : 1.0f / sqrtf((float)c.d_head);
+  d.plan_id = next_id.fetch_add(1);
+  if (d.plan_id == 0) d.plan_id = next_id.fetch_add(1);
   d.nchunk_per_head = (int32_t)((N + kChunk - 1) / kChunk);
   if (c.mode == HTTM_DENSE) {
     d.max_items = (int32_t)(c.h * ((N + kAttnRows - 1) / kAttnRows));
@@ -502,6 +510,11 @@ httm_status httm_forward_with_plan(httm_plan_t plan, const void* Q, const void* 
                                    const httm_debug* dbg, void* stream) {
   if (!injected) return HTTM_ERR_ARG;
   return forward_impl(plan, Q, K, V, out, workspace, workspace_bytes, injected, dbg, stream);
+}
+
+httm_status httm_forward_reuse(httm_plan_t plan, const void* Q, const void* K, const void* V, void* out,
+                               void* workspace, size_t workspace_bytes, void* stream) {
+  return forward_impl(plan, Q, K, V, out, workspace, workspace_bytes, nullptr, nullptr, stream, true);
 }
 
 httm_status httm_reorder(httm_plan_t plan, const void* X, void* Xb, int inverse, void* stream) {

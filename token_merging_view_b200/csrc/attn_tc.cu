@@ -252,7 +252,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         rsum = ((r0 + r1) + (r2 + r3)) + ((r4 + r5) + (r6 + r7));
         if (pass == 1) break;
         const float mts = max3(mx[0], mx[1], fmaxf(mx[2], mx[3])) * scale_log2;
-        const bool need = mts > m_used + 8.f;
+        // rows past the item's end (padding, or the next head's rows) hold
+        // whatever the buffer holds: they never ask for a redo, so that the
+        // live rows' results do not depend on them
+        const bool need = t * kBM + row < n_rows && mts > m_used + 8.f;
         if (!__any_sync(0xffffffffu, need)) break;
         const float m_new = fmaxf(m_used, mts);
         const float alpha = ex2(m_used - m_new);

@@ -37,6 +37,7 @@ struct Dims {
   int32_t nchunk_per_head;       // chunks of the outlier scan per head
   int32_t max_items;             // attention work items (upper bound)
   float scale;
+  uint32_t plan_id;              // stamps a workspace whose member lists this plan wrote
 };
 
 constexpr int kChunk = 4096;       // keys per chunk of the outlier compaction
@@ -48,14 +49,14 @@ struct DevState {
   uint32_t status;               // HTTM_DEV_* bits (sticky until read)
   uint32_t n_eligible;           // queries in groups of >= 2 tokens
   uint32_t n_items;              // live attention work items
-  uint32_t pad0;
+  uint32_t plan_stamp;           // plan_id of the member lists held (0: none)
   uint32_t sel[8];               // outlier select: threshold key, eq budget, total
 };
 
 struct Workspace {
   size_t state, hist, chunk, n_out, out_base, items;
   size_t q_best, q_score, q_merged, k_best, k_score, k_merged;
-  size_t q_slot, keys, mask, q_members, q_gstart, q_gcount, k_members, k_gstart, k_gcount;
+  size_t q_slot, q_orank, keys, mask, q_members, q_gstart, q_gcount, k_members, k_gstart, k_gcount;
   size_t q_tilde, k_tilde, v_tilde, o_tilde;
   size_t total;
 };
@@ -72,7 +73,8 @@ struct Buffers {
   int4* items;             // [max_items]: head, q_row0, n_rows, unused
   int32_t* q_best; float* q_score; uint8_t* q_merged;
   int32_t* k_best; float* k_score; uint8_t* k_merged;
-  int32_t* q_slot;         // [h, N]
+  int32_t* q_slot;         // [h, N]: regular query slot of every token (kept across calls)
+  int32_t* q_orank;        // [h, N]: rank of an outlier within its head (valid where mask is set)
   uint32_t* keys;          // [h, N]: eligible ? bits(dev) + 1 : 0
   uint8_t* mask;           // [h, N]
   int32_t* q_members;      // [h, N]: tokens in slot order (block after block)

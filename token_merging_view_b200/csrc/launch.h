@@ -21,7 +21,9 @@ struct Inject {
   const uint8_t* outlier;
 };
 
-cudaError_t launch_zero_state(const Dims& dims, const Buffers& buf, cudaStream_t s);
+// Clears the per-call state; `keep_stamp` keeps the record of which plan
+// wrote the workspace's member lists (calls that reuse them).
+cudaError_t launch_zero_state(const Dims& dims, const Buffers& buf, bool keep_stamp, cudaStream_t s);
 
 cudaError_t launch_match_simt(const Dims& dims, bool fp32, const BlockDesc* blocks,
                               const int4* items, int n_items, const void* Q, const void* K,
@@ -37,8 +39,9 @@ cudaError_t launch_import_plan(const Dims& dims, const BlockDesc* blocks, const 
                                const Buffers& buf, cudaStream_t s);
 
 // Merge planning (Q and K) then the mean-merging gathers of Q and of K/V:
-// three launches.
-cudaError_t launch_merge(const Dims& dims, bool fp32, const BlockDesc* blocks, bool injected,
+// three launches; with `reuse`, only the gathers, on the member lists an
+// earlier call left in the workspace.
+cudaError_t launch_merge(const Dims& dims, bool fp32, const BlockDesc* blocks, bool injected, bool reuse,
                          const void* Q, const void* K, const void* V, const Buffers& buf,
                          const Debug& dbg, cudaStream_t s);
 

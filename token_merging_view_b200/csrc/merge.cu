@@ -377,12 +377,16 @@ plan_kernel(Dims dims, const BlockDesc* __restrict__ blocks, Buffers buf, Debug 
 // keys is histogrammed for the global outlier select.
 template <class T, int D, bool IS_Q>
 __global__ void __launch_bounds__(256)
-gather_kernel(Dims dims, const T* __restrict__ X, const T* __restrict__ V, Buffers buf, Debug dbg) {
+gather_kernel(Dims dims, const T* __restrict__ X, const T* __restrict__ V, Buffers buf, Debug dbg, int reuse) {
   using Ch = Chunk<T, D>;
   constexpr int CPR = Ch::CPR, RPI = Ch::RPI, EPC = Ch::EPC, kU = 4;
   __shared__ uint32_t hist[IS_Q ? kHistBins : 1];
   __shared__ uint32_t s_elig;
+  // member lists from an earlier call must carry this plan's stamp
+  if (reuse && threadIdx.x == 0 && *(volatile uint32_t*)&buf.state->plan_stamp != dims.plan_id)
+    set_status(buf.state, HTTM_DEV_BAD_PLAN);
   if (cta_plan_failed(buf.state)) return;
+  if (!reuse && IS_Q && blockIdx.x == 0 && threadIdx.x == 0) buf.state->plan_stamp = dims.plan_id;
   const int tid = threadIdx.x, lane = tid & 31;
   const int rg = lane / CPR, ch = lane % CPR;
   if (IS_Q) {
@@ -661,7 +665,7 @@ __global__ void export_kernel(Dims dims, const BlockDesc* __restrict__ blocks, B
       if (os) os[idx] = sc;
       if (om) om[idx] = (uint8_t)mg;
     }
-    if (dbg.q_slot) dbg.q_slot[idx] = buf.q_slot[idx];
+    if (dbg.q_slot) dbg.q_slot[idx] = buf.mask[idx] ? dims.q_slots + buf.q_orank[idx] : buf.q_slot[idx];
     if (dbg.dev) {
       const uint32_t key = buf.keys[idx];
       dbg.dev[idx] = key ? __uint_as_float(key - 1u) : 0.f;
@@ -670,9 +674,10 @@ __global__ void export_kernel(Dims dims, const BlockDesc* __restrict__ blocks, B
   }
 }
 
-__global__ void zero_state_kernel(Buffers buf) {
+__global__ void zero_state_kernel(Buffers buf, int keep_stamp) {
   for (int i = threadIdx.x; i < 3 * kHistBins; i += blockDim.x) buf.hist[i] = 0u;
   if (threadIdx.x == 0) {
+    if (!keep_stamp) buf.state->plan_stamp = 0u;   // rewritten once this call's planning has succeeded
     buf.state->status = 0u;
     buf.state->n_eligible = 0u;
     buf.state->n_items = 0u;
@@ -685,37 +690,41 @@ int gather_grid(long long units) {
 }
 
 template <class T, int D>
-cudaError_t launch_merge_t(const Dims& dims, const BlockDesc* blocks, bool injected, const void* Q, const void* K,
-                           const void* V, const Buffers& buf, const Debug& dbg, cudaStream_t s) {
-  const int cap = (dims.max_nsrc + kMergeThreads - 1) / kMergeThreads * kMergeThreads;
-  const size_t smem = (size_t)cap * 13 + 3ull * dims.max_ndst * 4 + (size_t)kHistBins * 4 + 64 * 4;
-  cudaError_t e = cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  plan_kernel<<<dim3(dims.nblk, dims.h, 2), kMergeThreads, smem, s>>>(dims, blocks, buf, dbg, injected ? 1 : 0, cap);
+cudaError_t launch_merge_t(const Dims& dims, const BlockDesc* blocks, bool injected, bool reuse, const void* Q,
+                           const void* K, const void* V, const Buffers& buf, const Debug& dbg, cudaStream_t s) {
+  if (!reuse) {
+    const int cap = (dims.max_nsrc + kMergeThreads - 1) / kMergeThreads * kMergeThreads;
+    const size_t smem = (size_t)cap * 13 + 3ull * dims.max_ndst * 4 + (size_t)kHistBins * 4 + 64 * 4;
+    cudaError_t e = cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    plan_kernel<<<dim3(dims.nblk, dims.h, 2), kMergeThreads, smem, s>>>(dims, blocks, buf, dbg, injected ? 1 : 0,
+                                                                        cap);
+  }
   constexpr int RPI = Chunk<T, D>::RPI;
   // resident warps handle several slots each, so that prefetching pays
   gather_kernel<T, D, true><<<gather_grid((long long)dims.h * dims.q_slots / (4 * RPI) + 1), 256, 0, s>>>(
-      dims, (const T*)Q, nullptr, buf, dbg);
+      dims, (const T*)Q, nullptr, buf, dbg, reuse ? 1 : 0);
   gather_kernel<T, D, false><<<gather_grid((long long)dims.h * dims.k_slots / (4 * RPI) + 1), 256, 0, s>>>(
-      dims, (const T*)K, (const T*)V, buf, dbg);
+      dims, (const T*)K, (const T*)V, buf, dbg, reuse ? 1 : 0);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_zero_state(const Dims&, const Buffers& buf, cudaStream_t s) {
-  zero_state_kernel<<<1, 1024, 0, s>>>(buf);
+cudaError_t launch_zero_state(const Dims&, const Buffers& buf, bool keep_stamp, cudaStream_t s) {
+  zero_state_kernel<<<1, 1024, 0, s>>>(buf, keep_stamp ? 1 : 0);
   return cudaGetLastError();
 }
 
-cudaError_t launch_merge(const Dims& dims, bool fp32, const BlockDesc* blocks, bool injected, const void* Q,
-                         const void* K, const void* V, const Buffers& buf, const Debug& dbg, cudaStream_t s) {
+cudaError_t launch_merge(const Dims& dims, bool fp32, const BlockDesc* blocks, bool injected, bool reuse,
+                         const void* Q, const void* K, const void* V, const Buffers& buf, const Debug& dbg,
+                         cudaStream_t s) {
   if (fp32) {
-    if (dims.d == 16) return launch_merge_t<float, 16>(dims, blocks, injected, Q, K, V, buf, dbg, s);
-    return launch_merge_t<float, 64>(dims, blocks, injected, Q, K, V, buf, dbg, s);
+    if (dims.d == 16) return launch_merge_t<float, 16>(dims, blocks, injected, reuse, Q, K, V, buf, dbg, s);
+    return launch_merge_t<float, 64>(dims, blocks, injected, reuse, Q, K, V, buf, dbg, s);
   }
-  if (dims.d == 16) return launch_merge_t<__nv_bfloat16, 16>(dims, blocks, injected, Q, K, V, buf, dbg, s);
-  return launch_merge_t<__nv_bfloat16, 64>(dims, blocks, injected, Q, K, V, buf, dbg, s);
+  if (dims.d == 16) return launch_merge_t<__nv_bfloat16, 16>(dims, blocks, injected, reuse, Q, K, V, buf, dbg, s);
+  return launch_merge_t<__nv_bfloat16, 64>(dims, blocks, injected, reuse, Q, K, V, buf, dbg, s);
 }
 
 cudaError_t launch_restore(const Dims& dims, bool fp32, const BlockDesc*, const void* Q, const Buffers& buf,

@@ -27,54 +27,58 @@ __device__ __forceinline__ uint32_t k_total(const Dims& dims, const Buffers& buf
   return (uint32_t)min((unsigned long long)dims.k_out_max, e);
 }
 
-// One full warp: the bin holding the k-th largest key (k >= 1) of hist[0, nb)
-// and k minus the number of keys in higher bins.
-__device__ void select_bin(const uint32_t* hist, int nb, uint32_t k, int* bin, uint32_t* krem) {
-  const int lane = threadIdx.x & 31;
-  uint32_t above = 0;
-  for (int top = nb - 1; top >= 0; top -= 32) {
-    const int bb = top - lane;
-    const uint32_t c = bb >= 0 ? hist[bb] : 0u;
-    const uint32_t inc = warp_incl_scan(c);
-    const uint32_t tot = __shfl_sync(0xffffffffu, inc, 31);
-    if (above + tot >= k) {
-      const unsigned ballot = __ballot_sync(0xffffffffu, above + inc >= k);
-      const int l = __ffs(ballot) - 1;
-      const uint32_t inc_l = __shfl_sync(0xffffffffu, inc, l);
-      const uint32_t c_l = __shfl_sync(0xffffffffu, c, l);
-      *bin = top - l;
-      *krem = k - (above + inc_l - c_l);
-      return;
-    }
-    above += tot;
-  }
-  *bin = 0;
-  *krem = 0;
-}
-
 // Selected digits of the passes done so far (computed by warp 0 of each CTA).
 struct Sel {
   int b1, b2, b3;
   uint32_t k1, k2, k3;
 };
 
-__device__ void select_digits(const Buffers& buf, uint32_t k, int passes, Sel* s) {
-  if ((threadIdx.x >> 5) != 0) return;
-  select_bin(buf.hist, kHistBins, k, &s->b1, &s->k1);
-  if (passes >= 2) select_bin(buf.hist + kHistBins, kHistBins, s->k1, &s->b2, &s->k2);
-  if (passes >= 3) select_bin(buf.hist + 2 * kHistBins, 1024, s->k2, &s->b3, &s->k3);
+// The bin holding the k-th largest key of hist[0, nb) by the whole block
+// (each thread owns nb / blockDim.x consecutive bins from the top; one block
+// scan finds the owner), and k minus the keys in higher bins.
+__device__ void block_select(const uint32_t* hist, int nb, uint32_t k, uint32_t* tmp, int* bin, uint32_t* krem) {
+  const int per = nb / blockDim.x;
+  const int top = nb - 1 - threadIdx.x * per;
+  if (threadIdx.x == 0) {   // k above the histogram's total: bin 0 (the owner, if any, writes after the scan)
+    *bin = 0;
+    *krem = 0;
+  }
+  uint32_t s = 0;
+  for (int i = 0; i < per; ++i) s += hist[top - i];
+  uint32_t tot;
+  uint32_t above = block_excl_scan(s, tmp, &tot);
+  if (above < k && k <= above + s) {
+    for (int i = 0; i < per; ++i) {
+      const uint32_t c = hist[top - i];
+      if (k <= above + c) {
+        *bin = top - i;
+        *krem = k - above;
+        break;
+      }
+      above += c;
+    }
+  }
+  __syncthreads();
+}
+
+// Selected digits of the passes done so far, by every thread of the block
+// (blockDim.x = 1024).
+__device__ void select_digits(const Buffers& buf, uint32_t k, int passes, Sel* s, uint32_t* tmp) {
+  block_select(buf.hist, kHistBins, k, tmp, &s->b1, &s->k1);
+  if (passes >= 2) block_select(buf.hist + kHistBins, kHistBins, s->k1, tmp, &s->b2, &s->k2);
+  if (passes >= 3) block_select(buf.hist + 2 * kHistBins, 1024, s->k2, tmp, &s->b3, &s->k3);
 }
 
 // Histogram of the next digit among keys whose higher digits were selected.
 __global__ void __launch_bounds__(1024) hist_pass_kernel(Dims dims, Buffers buf, int pass) {
   __shared__ uint32_t sh[kHistBins];
   __shared__ Sel sel;
+  __shared__ uint32_t tmp[40];
   if (cta_plan_failed(buf.state)) return;
   const uint32_t k = k_total(dims, buf);
   if (k == 0) return;
   for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sh[i] = 0u;
-  select_digits(buf, k, pass - 1, &sel);
-  __syncthreads();
+  select_digits(buf, k, pass - 1, &sel, tmp);
   const size_t total = (size_t)dims.h * dims.N;
   const uint32_t pre = pass == 2 ? (uint32_t)sel.b1 : ((uint32_t)sel.b1 << 11) | (uint32_t)sel.b2;
   const int shift = pass == 2 ? 21 : 10;
@@ -101,8 +105,7 @@ __global__ void __launch_bounds__(1024) out_count_kernel(Dims dims, Buffers buf,
   const uint32_t k = k_total(dims, buf);
   if (!mask_injected) {
     if (k > 0) {
-      select_digits(buf, k, 3, &sel);
-      __syncthreads();
+      select_digits(buf, k, 3, &sel, tmp);
       T = ((uint32_t)sel.b1 << 21) | ((uint32_t)sel.b2 << 10) | (uint32_t)sel.b3;
       need = sel.k3;
       for (int n = lo + threadIdx.x; n < hi; n += blockDim.x) {
@@ -265,7 +268,7 @@ out_emit_kernel(Dims dims, const T* __restrict__ Q, Buffers buf, int mask_inject
     if (n >= hi) continue;
     buf.mask[base + n] = out[j] ? 1 : 0;
     if (out[j]) {
-      buf.q_slot[base + n] = dims.q_slots + (int32_t)rank;
+      buf.q_orank[base + n] = (int32_t)rank;
       const T* src = Qh + (size_t)n * D;
       T* dst = Qt + ((size_t)buf.out_base[hh] + rank) * D;
       constexpr int VEC = (int)(D * sizeof(T) / 16);

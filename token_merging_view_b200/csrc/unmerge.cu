@@ -27,7 +27,7 @@ unmerge_kernel(Dims dims, const uint4* __restrict__ Ot, uint4* __restrict__ out,
     const size_t tok = i / VEC;
     const int v = (int)(i - tok * VEC);
     const int hh = (int)(tok / dims.N);
-    const int32_t s = buf.q_slot[tok];
+    const int32_t s = buf.mask[tok] ? dims.q_slots + buf.q_orank[tok] : buf.q_slot[tok];
     size_t row;
     if (s < dims.q_slots) row = (size_t)hh * dims.q_slots + s;
     else row = (size_t)buf.out_base[hh] + (s - dims.q_slots);
