@@ -31,10 +31,12 @@
 // sub-partition busy on the exp unit while the tensor core alternates
 // between the tiles.
 //
-// Softmax: base-2 running max, updated lazily -- O_t and the row sum are
-// rescaled only when the row max grows by more than 8 (log2 units), so P stays
-// below 2^8 and most tiles never touch O_t; max and sum use split
-// accumulators for instruction-level parallelism.  Every wait is bounded
+// Softmax: base-2 max, updated lazily -- the exponentials of a tile are taken
+// against the max in use, and O_t and the row sum are rescaled (and the tile
+// redone) only when they sum above 2^16, i.e. when some score lies more than
+// 16 log2 units above that max; P stays below 2^16 and most tiles never touch
+// O_t nor compute a max.  Sums use split accumulators for instruction-level
+// parallelism.  Every wait is bounded
 // (2 s): a wait that runs out sets HTTM_DEV_TIMEOUT, the CTA drains its MMAs,
 // frees TMEM and exits.
 #include <mutex>
@@ -211,30 +213,26 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         for (int i = 0; i < kBN; ++i)
           if (i >= valid) sr[i] = __float_as_uint(-INFINITY);
       }
-      // p = 2^(s * c - m) with the running max m as it stands: the affine
-      // part and the row sums on packed fp32 pairs, the exponentials on the
-      // exp unit, and the tile max tracked alongside (three-input max).  If a
-      // row's tile max exceeds m by more than 8 (log2 units) -- always on
-      // the first tile, rarely afterwards -- the warp rescales O and the sum
-      // and redoes the tile with the new max.
+      // p = 2^(s * c - m) with the max m in use: the affine part and the row
+      // sums on packed fp32 pairs, the exponentials on the exp unit.  A row
+      // whose exponentials sum above 2^16 has a score more than 16 (log2
+      // units) above m -- always so on the first tile, where m = -inf --
+      // and makes the warp rescale O and the sum to the row's new max and
+      // redo the tile.  Otherwise P stays below 2^16 and O_t is untouched.
       const unsigned long long cc = f2_pack(scale_log2, scale_log2);
+      const bool live_row = t * kBM + row < n_rows;
       float rsum = 0.f;
       for (int pass = 0; pass < 2; ++pass) {
         const unsigned long long mm = f2_pack(-m_used, -m_used);
         unsigned long long rs[4];
-        float mx[4];
 #pragma unroll
-        for (int a = 0; a < 4; ++a) {
-          rs[a] = 0ull;                                  // (0.f, 0.f)
-          mx[a] = -INFINITY;
-        }
+        for (int a = 0; a < 4; ++a) rs[a] = 0ull;         // (0.f, 0.f)
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           uint32_t pk[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const float s0 = __uint_as_float(sr[c * 64 + 2 * i]), s1 = __uint_as_float(sr[c * 64 + 2 * i + 1]);
-            mx[i & 3] = max3(mx[i & 3], s0, s1);
             const unsigned long long xp = f2_fma(f2_pack(s0, s1), cc, mm);
             float x0, x1;
             f2_unpack(xp, x0, x1);
@@ -251,12 +249,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         f2_unpack(rs[3], r6, r7);
         rsum = ((r0 + r1) + (r2 + r3)) + ((r4 + r5) + (r6 + r7));
         if (pass == 1) break;
-        const float mts = max3(mx[0], mx[1], fmaxf(mx[2], mx[3])) * scale_log2;
         // rows past the item's end (padding, or the next head's rows) hold
         // whatever the buffer holds: they never ask for a redo, so that the
-        // live rows' results do not depend on them
-        const bool need = t * kBM + row < n_rows && mts > m_used + 8.f;
+        // live rows' results do not depend on them.  NaN sums (the first
+        // tile's masked tail) count as large.
+        const bool need = live_row && !(rsum <= 65536.f);
         if (!__any_sync(0xffffffffu, need)) break;
+        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int i = 0; i < 64; ++i)
+          mx[i & 3] = max3(mx[i & 3], __uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1]));
+        const float mts = max3(mx[0], mx[1], fmaxf(mx[2], mx[3])) * scale_log2;
         const float m_new = fmaxf(m_used, mts);
         const float alpha = ex2(m_used - m_new);
         if (j > 0) {
