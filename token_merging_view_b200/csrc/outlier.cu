@@ -196,19 +196,22 @@ __global__ void __launch_bounds__(1024) out_scan_kernel(Dims dims, Buffers buf) 
     buf.state->sel[3] = (uint32_t)total;
   }
   __syncthreads();
+  // head after head: its regular slot tiles, then its outlier tiles, so
+  // that the CTAs reading one head's K~/V~ run close together in time and
+  // find them in L2
   const int tq = (dims.q_slots + kAttnRows - 1) / kAttnRows;
-  const int nreg = dims.h * tq;
-  for (int i = tid; i < nreg; i += blockDim.x) {
+  for (int i = tid; i < dims.h * tq; i += blockDim.x) {
     const int hh = i / tq, t = i - hh * tq;
-    buf.items[i] = make_int4(hh, hh * dims.q_slots + t * kAttnRows, min(kAttnRows, dims.q_slots - t * kAttnRows), 0);
+    buf.items[hh * tq + tile_off[hh] + t] =
+        make_int4(hh, hh * dims.q_slots + t * kAttnRows, min(kAttnRows, dims.q_slots - t * kAttnRows), 0);
   }
   for (int hh = 0; hh < dims.h; ++hh) {
     const int nt = tile_off[hh + 1] - tile_off[hh];
     for (int t = tid; t < nt; t += blockDim.x)
-      buf.items[nreg + tile_off[hh] + t] =
+      buf.items[(hh + 1) * tq + tile_off[hh] + t] =
           make_int4(hh, buf.out_base[hh] + t * kAttnRows, min(kAttnRows, buf.n_out[hh] - t * kAttnRows), 0);
   }
-  if (tid == 0) buf.state->n_items = (uint32_t)(nreg + tile_off[dims.h]);
+  if (tid == 0) buf.state->n_items = (uint32_t)(dims.h * tq + tile_off[dims.h]);
 }
 
 // Per chunk: decide each query, write M_o, give outliers their slots and
