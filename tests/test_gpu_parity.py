@@ -159,6 +159,17 @@ def test_deterministic():
         assert np.array_equal(da[key], db[key], equal_nan=True), key
 
 
+@pytest.mark.parametrize("w", [MID, TINY, WORKLOADS["vggt_30f"]], ids=lambda w: w.name)
+def test_plain_and_debug_calls_agree(w):
+    """httm_forward restores only the slots holding outliers; the debug call
+    (which exports every slot's restored mean) walks all slots.  Same bits."""
+    _, plan, _, (Q, K, V), _ = _case(w)
+    a = B.httm_forward(plan, Q, K, V, workspace=plan.new_workspace())
+    b, _, _, status = PL.run(plan, Q, K, V)
+    assert status == 0
+    assert torch.equal(a, b)
+
+
 def test_output_independent_of_workspace_contents():
     """Rows of Q~ past a work item's end are never written; attention must
     not let them change the live rows (filled with zeros, then with large

@@ -107,6 +107,7 @@ Workspace layout(const Dims& d, bool fp32) {
   w.k_merged = take((size_t)d.h * d.k_src);
   w.q_slot = take(hN * 4);
   w.q_orank = take(hN * 4);
+  w.o_tok = take((size_t)(d.q_rows_alloc - d.out_base) * 4);
   w.keys = take(hN * 4);
   w.mask = take(hN);
   w.q_members = take(hN * 4);
@@ -140,6 +141,7 @@ Buffers resolve(const Workspace& w, void* base) {
   b.k_merged = reinterpret_cast<uint8_t*>(p + w.k_merged);
   b.q_slot = reinterpret_cast<int32_t*>(p + w.q_slot);
   b.q_orank = reinterpret_cast<int32_t*>(p + w.q_orank);
+  b.o_tok = reinterpret_cast<int32_t*>(p + w.o_tok);
   b.keys = reinterpret_cast<uint32_t*>(p + w.keys);
   b.mask = reinterpret_cast<uint8_t*>(p + w.mask);
   b.q_members = reinterpret_cast<int32_t*>(p + w.q_members);

@@ -56,7 +56,7 @@ struct DevState {
 struct Workspace {
   size_t state, hist, chunk, n_out, out_base, items;
   size_t q_best, q_score, q_merged, k_best, k_score, k_merged;
-  size_t q_slot, q_orank, keys, mask, q_members, q_gstart, q_gcount, k_members, k_gstart, k_gcount;
+  size_t q_slot, q_orank, o_tok, keys, mask, q_members, q_gstart, q_gcount, k_members, k_gstart, k_gcount;
   size_t q_tilde, k_tilde, v_tilde, o_tilde;
   size_t total;
 };
@@ -75,6 +75,7 @@ struct Buffers {
   int32_t* k_best; float* k_score; uint8_t* k_merged;
   int32_t* q_slot;         // [h, N]: regular query slot of every token (kept across calls)
   int32_t* q_orank;        // [h, N]: rank of an outlier within its head (valid where mask is set)
+  int32_t* o_tok;          // [q_rows_alloc - out_base]: token (within its head) of each outlier row of Q~
   uint32_t* keys;          // [h, N]: eligible ? bits(dev) + 1 : 0
   uint8_t* mask;           // [h, N]
   int32_t* q_members;      // [h, N]: tokens in slot order (block after block)

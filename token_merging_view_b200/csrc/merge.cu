@@ -23,6 +23,7 @@ namespace httm {
 namespace {
 
 constexpr int kMergeThreads = 256;
+static_assert(kMergeThreads == 256, "the planning kernel clears and selects 256 radix bins, one per thread");
 
 // A [D]-row spread over one warp: lane l owns elements [l*E, l*E + E).
 template <class T, int D>
@@ -180,22 +181,36 @@ __device__ void block_select_bin(const uint32_t* hist, int nb, uint32_t k, uint3
   __syncthreads();
 }
 
+// Quotient of n by d for n, d < 2^16 as a multiply-high by ceil(2^32 / d):
+// exact because n * d < 2^32 keeps the error of the product below 1 / d.
+struct SmallDiv {
+  unsigned long long m;
+  __device__ explicit SmallDiv(uint32_t d) : m(0xFFFFFFFFull / d + 1ull) {}
+  __device__ uint32_t div(uint32_t n) const { return (uint32_t)(((unsigned long long)n * m) >> 32); }
+};
+
 // Merge planning, one CTA per (block, head, tensor): which sources merge
 // (top-r), their groups, and the member lists (CSR) the gather kernel reads.
 // Members of a destination group: the destination, then its merged sources
 // by ascending in-block index; kept sources follow as singletons.  Every
-// token of the block is the member of exactly one slot.
+// token of the block is the member of exactly one slot.  Every phase is
+// spread evenly over the threads: the top-r threshold by a 4-digit radix
+// select (8-bit digits), group sizes by shared-memory counting, each merged
+// source's place in its group by counting the group's smaller ordinals, and
+// the member list written position by position (a binary search over the
+// group starts finds each position's group).
 __global__ void __launch_bounds__(kMergeThreads)
 plan_kernel(Dims dims, const BlockDesc* __restrict__ blocks, Buffers buf, Debug dbg, int injected, int cap) {
   extern __shared__ __align__(16) unsigned char smem[];
   uint32_t* key = reinterpret_cast<uint32_t*>(smem);        // [cap] ordered score bits
-  int32_t* mem = reinterpret_cast<int32_t*>(key + cap);      // [cap] merged by group, then kept
+  int32_t* bst = reinterpret_cast<int32_t*>(key + cap);      // [cap] destination of each source
+  int32_t* mem = bst + cap;                                  // [cap] merged by group, then kept
   int32_t* aux = mem + cap;                                  // [cap] merged, unordered within a group
   int32_t* cm = aux + cap;                                   // [max_ndst] merged sources per destination
   int32_t* gsm = cm + dims.max_ndst;                         // [max_ndst] exclusive scan of cm
   int32_t* cur = gsm + dims.max_ndst;                        // [max_ndst] placement cursors
-  uint32_t* rh = reinterpret_cast<uint32_t*>(cur + dims.max_ndst);  // [kHistBins] radix select
-  uint32_t* tmp = rh + kHistBins;                            // [64]
+  uint32_t* rh = reinterpret_cast<uint32_t*>(cur + dims.max_ndst);  // [256] radix select
+  uint32_t* tmp = rh + 256;                                  // [64]
   uint8_t* mf = reinterpret_cast<uint8_t*>(tmp + 64);        // [cap] merged flag
   __shared__ int s_bad;
   __shared__ int s_bin;
@@ -203,7 +218,6 @@ plan_kernel(Dims dims, const BlockDesc* __restrict__ blocks, Buffers buf, Debug 
 
   const bool is_q = blockIdx.z == 0;
   const int tid = threadIdx.x, bd = blockDim.x;
-  const int lane = tid & 31, warp = tid >> 5, nwarps = bd >> 5;
   const int hh = blockIdx.y;
   const BlockDesc b = blocks[blockIdx.x];
   const int stride = is_q ? dims.q_stride : dims.kv_stride;
@@ -227,29 +241,31 @@ plan_kernel(Dims dims, const BlockDesc* __restrict__ blocks, Buffers buf, Debug 
   if (cta_plan_failed(buf.state)) return;
   if (tid == 0) s_bad = 0;
   for (int m = tid; m < ndst; m += bd) cm[m] = 0;
+  for (int k = tid; k < nsrc; k += bd) {
+    bst[k] = best[k];
+    if (!injected) key[k] = float_order(score[k]);
+  }
+  __syncthreads();
 
   // 1. top-r: the r sources with the largest (score, -ordinal) merge.  The
-  //    r-th largest ordered score T comes from a 3-digit radix select; all
-  //    keys above T merge, and of the keys equal to T the lowest ordinals.
+  //    r-th largest ordered score T comes from the radix select; all keys
+  //    above T merge, and of the keys equal to T the lowest ordinals.
   if (!injected) {
-    for (int k = tid; k < nsrc; k += bd) key[k] = float_order(score[k]);
     uint32_t T = 0, need = 0;
     if (r > 0) {
       uint32_t prefix = 0, krem = (uint32_t)r;
 #pragma unroll 1
-      for (int pass = 0; pass < 3; ++pass) {
-        const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
-        const int nb = pass == 2 ? 1024 : 2048;
-        for (int i = tid; i < kHistBins; i += bd) rh[i] = 0;
+      for (int pass = 0; pass < 4; ++pass) {
+        const int shift = 24 - 8 * pass;
+        rh[tid] = 0;                                     // blockDim.x == 256 bins
         __syncthreads();
         for (int k = tid; k < nsrc; k += bd) {
           const uint32_t kk = key[k];
-          if (pass == 0 || (kk >> (shift + (pass == 1 ? 11 : 10))) == prefix)
-            atomicAdd(&rh[(kk >> shift) & (uint32_t)(nb - 1)], 1u);
+          if (pass == 0 || (kk >> (shift + 8)) == prefix) atomicAdd(&rh[(kk >> shift) & 255u], 1u);
         }
         __syncthreads();
-        block_select_bin(rh, nb, krem, tmp, &s_bin, &s_krem);
-        prefix = (prefix << (pass == 2 ? 10 : 11)) | (uint32_t)s_bin;
+        block_select_bin(rh, 256, krem, tmp, &s_bin, &s_krem);
+        prefix = (prefix << 8) | (uint32_t)s_bin;
         krem = s_krem;
       }
       T = prefix;
@@ -281,12 +297,12 @@ plan_kernel(Dims dims, const BlockDesc* __restrict__ blocks, Buffers buf, Debug 
   }
   __syncthreads();
 
-  // 2. groups: merged sources per destination (counting), placement, then
-  //    each group's members put in ascending ordinal by rank counting (the
-  //    placement order of atomics is not deterministic, the ranks are).
+  // 2. groups: merged sources per destination (counting), then placement
+  //    (in any order: atomics), then each merged source's place in its group
+  //    from the number of the group's smaller ordinals.
   for (int k = tid; k < nsrc; k += bd) {
     if (mf[k]) {
-      const int m = best[k];
+      const int m = bst[k];
       if (m < 0 || m >= ndst) s_bad = 1;
       else atomicAdd(&cm[m], 1);
     }
@@ -300,7 +316,7 @@ plan_kernel(Dims dims, const BlockDesc* __restrict__ blocks, Buffers buf, Debug 
   for (int m = tid; m < ndst; m += bd) cur[m] = gsm[m];
   __syncthreads();
   for (int k = tid; k < nsrc; k += bd)
-    if (mf[k]) aux[atomicAdd(&cur[best[k]], 1)] = k;
+    if (mf[k]) aux[atomicAdd(&cur[bst[k]], 1)] = k;
   {
     // kept sources in ascending ordinal after the r merged ones
     uint32_t nm = 0;
@@ -313,54 +329,51 @@ plan_kernel(Dims dims, const BlockDesc* __restrict__ blocks, Buffers buf, Debug 
     }
   }
   __syncthreads();
-  // small groups: one thread, insertion order; large groups: one warp, ranks
-  for (int m = tid; m < ndst; m += bd) {
-    const int s0 = gsm[m], c = cm[m];
-    if (c > 32) continue;
-    for (int i = 0; i < c; ++i) {
-      const int v = aux[s0 + i];
-      int j = i;
-      while (j > 0 && mem[s0 + j - 1] > v) {
-        mem[s0 + j] = mem[s0 + j - 1];
-        --j;
-      }
-      mem[s0 + j] = v;
-    }
-  }
-  for (int m = warp; m < ndst; m += nwarps) {
-    const int s0 = gsm[m], c = cm[m];
-    if (c <= 32) continue;
-    for (int i = lane; i < c; i += 32) {
-      const int v = aux[s0 + i];
-      int rank = 0;
-      for (int j = 0; j < c; ++j) rank += aux[s0 + j] < v;
-      mem[s0 + rank] = v;
-    }
+  for (int p = tid; p < r; p += bd) {
+    const int v = aux[p];
+    const int m = bst[v], s0 = gsm[m], c = cm[m];
+    int rank = 0;
+    for (int j = 0; j < c; ++j) rank += aux[s0 + j] < v;
+    mem[s0 + rank] = v;
   }
   __syncthreads();
 
-  // 3. member lists (tokens), slot starts and counts, the query slot map
+  // 3. member lists (tokens), slot starts and counts, the query slot map.
+  //    Group m holds positions [gsm[m] + m, gsm[m + 1] + m + 1); pm maps
+  //    each of those positions to m (key and bst are free by now and hold
+  //    2 * cap >= n_b entries).
+  int32_t* pm = reinterpret_cast<int32_t*>(key);
   for (int m = tid; m < ndst; m += bd) {
-    const int slot = slot_off + m;
-    const int pos = b.tok_off + gsm[m] + m;
-    const int c = cm[m] + 1;
-    for (int q = 0; q < c; ++q) {
-      const int tok = q == 0 ? block_token(b, m * stride, dims.P)
-                             : block_token(b, src_index(mem[gsm[m] + q - 1], stride), dims.P);
-      members[pos + q] = tok;
-      if (is_q) buf.q_slot[tokbase + tok] = slot;
-      else if (dbg.k_slot) dbg.k_slot[tokbase + tok] = slot;
-    }
-    gstart[slot] = pos;
-    gcount[slot] = c;
+    const int p0 = gsm[m] + m, c = cm[m] + 1;
+    gstart[slot_off + m] = b.tok_off + p0;
+    gcount[slot_off + m] = c;
+    for (int j = 0; j < c; ++j) pm[p0 + j] = m;
   }
   for (int p = tid; p < nsrc - r; p += bd) {
-    const int slot = slot_off + ndst + p;
-    const int pos = b.tok_off + ndst + r + p;
-    const int tok = block_token(b, src_index(mem[r + p], stride), dims.P);
-    members[pos] = tok;
-    gstart[slot] = pos;
-    gcount[slot] = 1;
+    gstart[slot_off + ndst + p] = b.tok_off + ndst + r + p;
+    gcount[slot_off + ndst + p] = 1;
+  }
+  __syncthreads();
+  const SmallDiv by_s(b.s), by_gap(stride - 1);
+  for (int q = tid; q < b.n_b; q += bd) {
+    int idx, slot;
+    if (q < ndst + r) {
+      const int a = pm[q], j = q - (gsm[a] + a);
+      if (j == 0) {
+        idx = a * stride;
+      } else {
+        const int k = mem[gsm[a] + j - 1], g = (int)by_gap.div(k);
+        idx = g * stride + (k - g * (stride - 1)) + 1;    // in-block index of source ordinal k
+      }
+      slot = slot_off + a;
+    } else {
+      const int p = q - ndst - r, k = mem[r + p], g = (int)by_gap.div(k);
+      idx = g * stride + (k - g * (stride - 1)) + 1;
+      slot = slot_off + ndst + p;
+    }
+    const int tau = (int)by_s.div(idx);
+    const int tok = b.base + tau * dims.P + (idx - tau * b.s);
+    members[b.tok_off + q] = tok;
     if (is_q) buf.q_slot[tokbase + tok] = slot;
     else if (dbg.k_slot) dbg.k_slot[tokbase + tok] = slot;
   }
@@ -376,7 +389,7 @@ plan_kernel(Dims dims, const BlockDesc* __restrict__ blocks, Buffers buf, Debug 
 // members of groups of >= 2, else 0), and the first radix digit of those
 // keys is histogrammed for the global outlier select.
 template <class T, int D, bool IS_Q>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 4)
 gather_kernel(Dims dims, const T* __restrict__ X, const T* __restrict__ V, Buffers buf, Debug dbg, int reuse) {
   using Ch = Chunk<T, D>;
   constexpr int CPR = Ch::CPR, RPI = Ch::RPI, EPC = Ch::EPC, kU = 4;
@@ -594,6 +607,98 @@ restore_kernel(Dims dims, const T* __restrict__ Q, Buffers buf, Debug dbg) {
   }
 }
 
+// Restore (key design 3) driven by the outliers: one row group per outlier
+// row of Q~ (rows [out_base, q_rows_alloc), head after head, with padding
+// between heads).  Of the outliers in one slot, the first in member order
+// recomputes the slot's mean from the remaining members -- the same members
+// in the same order, added the same way as the flat kernel above, so both
+// give the same bits; a slot whose members are all outliers is drained.
+template <class T, int D>
+__global__ void __launch_bounds__(256)
+restore_out_kernel(Dims dims, const T* __restrict__ Q, Buffers buf) {
+  using Ch = Chunk<T, D>;
+  constexpr int CPR = Ch::CPR, RPI = Ch::RPI, EPC = Ch::EPC, kU = 4;
+  __shared__ int s_base[64], s_nout[64];
+  if (plan_failed(buf.state)) return;
+  if (buf.state->sel[3] == 0) return;                 // no outlier anywhere
+  for (int i = threadIdx.x; i < dims.h; i += blockDim.x) {
+    s_base[i] = (int)(buf.out_base[i] - dims.out_base);
+    s_nout[i] = buf.n_out[i];
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int rg = lane / CPR, ch = lane % CPR;
+  const int span = (int)(dims.q_rows_alloc - dims.out_base);
+  T* Qt = reinterpret_cast<T*>(buf.q_tilde);
+  const int nwarp_total = gridDim.x * (blockDim.x >> 5);
+  for (int r0 = (blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * RPI; r0 < span; r0 += nwarp_total * RPI) {
+    const int row = r0 + rg;
+    int hh = -1;
+    if (row < span) {
+      for (int x = 0; x < dims.h; ++x)                 // row bases increase with the head
+        if (s_base[x] <= row) hh = x;
+      if (hh >= 0 && row - s_base[hh] >= s_nout[hh]) hh = -1;   // padding
+    }
+    int c = 0, gs = 0, gsl = 0, tok = -1;
+    size_t tokbase = 0;
+    if (hh >= 0) {
+      tokbase = (size_t)hh * dims.N;
+      tok = buf.o_tok[row];
+      const int sl = (tok >= 0 && tok < dims.N) ? buf.q_slot[tokbase + tok] : -1;
+      if (sl >= 0 && sl < dims.q_slots) {
+        gsl = hh * dims.q_slots + sl;
+        c = buf.q_gcount[gsl];
+        gs = buf.q_gstart[gsl];
+      }
+      if (c < 0 || gs < 0 || gs + c > dims.N || sl < 0 || sl >= dims.q_slots) {
+        if (ch == 0) set_status(buf.state, HTTM_DEV_BOUNDS);
+        c = 0;
+      }
+    }
+    // outliers among the members, and the first of them in member order
+    int nout = 0, first = 0x7fffffff;
+    for (int q = ch; q < c; q += CPR) {
+      const int m = buf.q_members[tokbase + gs + q];
+      const bool o = (m >= 0 && m < dims.N) && buf.mask[tokbase + m] != 0;
+      nout += o;
+      if (o && q < first) first = q;
+    }
+#pragma unroll
+    for (int o = 1; o < CPR; o <<= 1) {
+      nout += __shfl_xor_sync(0xffffffffu, nout, o);
+      first = min(first, __shfl_xor_sync(0xffffffffu, first, o));
+    }
+    const bool lead = c > 0 && first < c && buf.q_members[tokbase + gs + first] == tok;
+    const int cw = lead ? c : 0;
+    const int cmax = __reduce_max_sync(0xffffffffu, cw);
+    if (cmax == 0) continue;
+    float acc[EPC];
+#pragma unroll
+    for (int e = 0; e < EPC; ++e) acc[e] = 0.f;
+    for (int q0 = 0; q0 < cmax; q0 += kU) {
+      uint4 x[kU];
+      bool use[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        use[u] = false;
+        if (q0 + u < cw) {
+          const int m = buf.q_members[tokbase + gs + q0 + u];
+          use[u] = m >= 0 && m < dims.N && buf.mask[tokbase + m] == 0;
+          if (use[u]) x[u] = Ch::load(Q + (tokbase + m) * D, ch);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kU; ++u)
+        if (use[u]) Ch::add(acc, x[u]);
+    }
+    if (!lead) continue;
+    const int remain = c - nout;
+#pragma unroll
+    for (int e = 0; e < EPC; ++e) acc[e] = remain ? acc[e] / (float)remain : 0.f;
+    Ch::store(Qt + (size_t)gsl * D, ch, acc);
+  }
+}
+
 // Injected plan -> internal source-order arrays, with validation.
 __global__ void import_kernel(Dims dims, const BlockDesc* __restrict__ blocks, Inject inj, Buffers buf) {
   const size_t total = 2ull * dims.h * dims.N;
@@ -685,16 +790,20 @@ __global__ void zero_state_kernel(Buffers buf, int keep_stamp) {
   if (threadIdx.x < 8) buf.state->sel[threadIdx.x] = 0u;
 }
 
-int gather_grid(long long units) {
-  return (int)std::max<long long>(1, std::min<long long>((units + 7) / 8, 148 * 8));
+// CTAs of 8 warps for `units` warp-sized pieces of work, at most `per_sm`
+// per SM (the gathers run four per SM at their register bound; each warp
+// then takes several slots in turn, so that its prefetches pay).
+int gather_grid(long long units, int per_sm = 8) {
+  return (int)std::max<long long>(1, std::min<long long>((units + 7) / 8, 148LL * per_sm));
 }
 
 template <class T, int D>
 cudaError_t launch_merge_t(const Dims& dims, const BlockDesc* blocks, bool injected, bool reuse, const void* Q,
                            const void* K, const void* V, const Buffers& buf, const Debug& dbg, cudaStream_t s) {
   if (!reuse) {
-    const int cap = (dims.max_nsrc + kMergeThreads - 1) / kMergeThreads * kMergeThreads;
-    const size_t smem = (size_t)cap * 13 + 3ull * dims.max_ndst * 4 + (size_t)kHistBins * 4 + 64 * 4;
+    // cap sources per block, and 2 * cap >= n_b for the position map
+    const int cap = (std::max(dims.max_nsrc, (dims.max_nb + 1) / 2) + kMergeThreads - 1) / kMergeThreads * kMergeThreads;
+    const size_t smem = (size_t)cap * 17 + 3ull * dims.max_ndst * 4 + 256 * 4 + 64 * 4;
     cudaError_t e = cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     plan_kernel<<<dim3(dims.nblk, dims.h, 2), kMergeThreads, smem, s>>>(dims, blocks, buf, dbg, injected ? 1 : 0,
@@ -702,9 +811,9 @@ cudaError_t launch_merge_t(const Dims& dims, const BlockDesc* blocks, bool injec
   }
   constexpr int RPI = Chunk<T, D>::RPI;
   // resident warps handle several slots each, so that prefetching pays
-  gather_kernel<T, D, true><<<gather_grid((long long)dims.h * dims.q_slots / (4 * RPI) + 1), 256, 0, s>>>(
+  gather_kernel<T, D, true><<<gather_grid((long long)dims.h * dims.q_slots / (4 * RPI) + 1, 4), 256, 0, s>>>(
       dims, (const T*)Q, nullptr, buf, dbg, reuse ? 1 : 0);
-  gather_kernel<T, D, false><<<gather_grid((long long)dims.h * dims.k_slots / (4 * RPI) + 1), 256, 0, s>>>(
+  gather_kernel<T, D, false><<<gather_grid((long long)dims.h * dims.k_slots / (4 * RPI) + 1, 4), 256, 0, s>>>(
       dims, (const T*)K, (const T*)V, buf, dbg, reuse ? 1 : 0);
   return cudaGetLastError();
 }
@@ -729,20 +838,24 @@ cudaError_t launch_merge(const Dims& dims, bool fp32, const BlockDesc* blocks, b
 
 cudaError_t launch_restore(const Dims& dims, bool fp32, const BlockDesc*, const void* Q, const Buffers& buf,
                            const Debug& dbg, cudaStream_t s) {
-  const long long units = (long long)dims.h * dims.q_slots;
+  // the fp32 export needs every slot's restored mean: the flat kernel;
+  // otherwise only the slots holding outliers change
+  const bool flat = dbg.q_restored != nullptr;
+  const long long units = flat ? (long long)dims.h * dims.q_slots : dims.q_rows_alloc - dims.out_base;
+#define HTTM_RESTORE(T, DD)                                                                                  \
+  do {                                                                                                       \
+    const int grid = gather_grid(units / Chunk<T, DD>::RPI + 1);                                             \
+    if (flat) restore_kernel<T, DD><<<grid, 256, 0, s>>>(dims, (const T*)Q, buf, dbg);                       \
+    else restore_out_kernel<T, DD><<<grid, 256, 0, s>>>(dims, (const T*)Q, buf);                             \
+  } while (0)
   if (fp32) {
-    if (dims.d == 16)
-      restore_kernel<float, 16><<<gather_grid(units / Chunk<float, 16>::RPI + 1), 256, 0, s>>>(dims, (const float*)Q, buf, dbg);
-    else
-      restore_kernel<float, 64><<<gather_grid(units / Chunk<float, 64>::RPI + 1), 256, 0, s>>>(dims, (const float*)Q, buf, dbg);
+    if (dims.d == 16) HTTM_RESTORE(float, 16);
+    else HTTM_RESTORE(float, 64);
   } else {
-    if (dims.d == 16)
-      restore_kernel<__nv_bfloat16, 16><<<gather_grid(units / Chunk<__nv_bfloat16, 16>::RPI + 1), 256, 0, s>>>(
-          dims, (const __nv_bfloat16*)Q, buf, dbg);
-    else
-      restore_kernel<__nv_bfloat16, 64><<<gather_grid(units / Chunk<__nv_bfloat16, 64>::RPI + 1), 256, 0, s>>>(
-          dims, (const __nv_bfloat16*)Q, buf, dbg);
+    if (dims.d == 16) HTTM_RESTORE(__nv_bfloat16, 16);
+    else HTTM_RESTORE(__nv_bfloat16, 64);
   }
+#undef HTTM_RESTORE
   return cudaGetLastError();
 }
 

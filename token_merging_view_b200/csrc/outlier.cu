@@ -272,6 +272,7 @@ out_emit_kernel(Dims dims, const T* __restrict__ Q, Buffers buf, int mask_inject
     buf.mask[base + n] = out[j] ? 1 : 0;
     if (out[j]) {
       buf.q_orank[base + n] = (int32_t)rank;
+      buf.o_tok[(size_t)buf.out_base[hh] + rank - dims.out_base] = n;
       const T* src = Qh + (size_t)n * D;
       T* dst = Qt + ((size_t)buf.out_base[hh] + rank) * D;
       constexpr int VEC = (int)(D * sizeof(T) / 16);
