@@ -8,17 +8,22 @@
 // argmax_t dot(s, t) / ||t||, score = that / ||s||, so the n_src x n_dst
 // similarity matrix never leaves the SM.
 //
-// One CTA per (tensor, head, block, run of 128-source tiles), 9 warps:
-//   warps 0..7  gather rows with cp.async into the 128-byte-swizzled operand
+// One CTA per (tensor, head, block, run of 128-source tiles), 17 warps:
+//   warps 0..15 gather rows with cp.async into the 128-byte-swizzled operand
 //               layout (all destinations of the block once, then source tiles
 //               double-buffered), compute norms, and run the epilogue: warp w
 //               reads TMEM lanes 32*(w%4).. (one source row per thread) and the
-//               column half w/4 of each chunk; running (max, first index);
-//   warp 8      allocates TMEM and one thread issues tcgen05.mma: for each
+//               32-column groups g = w/4, w/4 + 4, ... of each chunk (both of
+//               its loads in flight at once); running (max, first index).
+//               Four warps per TMEM lane quarter keep the argmax, the bound of
+//               this kernel (a multiply, compare and two selects per score),
+//               issuing while others wait on TMEM or the MMA;
+//   warp 16     allocates TMEM and one thread issues tcgen05.mma: for each
 //               source tile, destination chunks of <= 256 columns into two
 //               TMEM buffers of 256 fp32 columns.
 // Ties keep the lowest destination (strict '>' in ascending column order;
-// the lower column half wins equal values).  Every wait is bounded.
+// of the four column parts the lowest index wins equal values).  Every wait
+// is bounded.
 #include "common.cuh"
 #include "launch.h"
 #include "tc_ptx.cuh"
@@ -28,7 +33,8 @@ namespace {
 
 using namespace tc;
 
-constexpr int kEpiThreads = 256;
+constexpr int kEpiThreads = 512;
+constexpr int kParts = kEpiThreads / 128;  // epilogue warps per TMEM lane quarter
 constexpr int kThreads = kEpiThreads + 32;
 constexpr int kMaxDst = 1024;          // destination rows a block may have on this path
 constexpr int kChunkCols = 256;
@@ -39,8 +45,8 @@ struct MatchSmem {
   uint8_t dst[kMaxDst * 128];          // K-major SW128, 128 KB
   uint8_t src[2][kTileBytes];
   float inv_d[kMaxDst];
-  float best_v[2][128];
-  int best_i[2][128];
+  float best_v[kParts][128];
+  int best_i[kParts][128];
   uint64_t src_ready[2], full[2], empty[2], drain;
   uint32_t tmem_base;
   int abort;
@@ -100,14 +106,14 @@ match_tc_kernel(Dims dims, const BlockDesc* __restrict__ blocks, const int4* __r
     sm.abort = 0;
     mbar_fence_init();
   }
-  if (warp == 8) tmem_alloc(&sm.tmem_base, 512);
+  if (warp == kEpiThreads / 32) tmem_alloc(&sm.tmem_base, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
   volatile int* abort = &sm.abort;
 
-  if (warp == 8) {
+  if (warp == kEpiThreads / 32) {
     if (lane == 0) {
       // ------------------------------------------------------------ MMA issue
       uint32_t gc = 0;
@@ -155,7 +161,7 @@ match_tc_kernel(Dims dims, const BlockDesc* __restrict__ blocks, const int4* __r
     };
     load_tile(0);
     cp_async_commit();
-    const int quarter = warp & 3, half = warp >> 2;
+    const int quarter = warp & 3, part = warp >> 2;
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     // Abort handling: a failed wait clears `ok` (warp-uniform) and sets the
@@ -192,9 +198,10 @@ match_tc_kernel(Dims dims, const BlockDesc* __restrict__ blocks, const int4* __r
         epi_sync();
       }
       mbar_arrive(&sm.src_ready[t & 1]);
-      // this row's inverse norm
-      float inv_s;
-      {
+      // this row's inverse norm (used by the warps of column part 0, which
+      // write the row's result)
+      float inv_s = 0.f;
+      if (part == 0) {
         float ss = 0.f;
         for (int ch = 0; ch < 8; ++ch) {
           const uint4 w = *reinterpret_cast<const uint4*>(sm.src[t & 1] + swz(row, ch));
@@ -208,8 +215,10 @@ match_tc_kernel(Dims dims, const BlockDesc* __restrict__ blocks, const int4* __r
         }
         inv_s = ss > 0.f ? 1.f / sqrtf(ss) : 0.f;
       }
-      float best = -INFINITY;
-      int bi = 0;
+      // four running (max, first index) pairs, one per column position mod 4
+      // (independent chains), merged below: larger value, lower index
+      float bv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      int bx[4] = {0x7fffffff, 0x7fffffff, 0x7fffffff, 0x7fffffff};
       for (int c = 0; c < nchunk; ++c, ++gc) {
         const uint32_t bb = gc & 1;
         if (ok && !__all_sync(0xffffffffu, mbar_wait(&sm.full[bb], (gc >> 1) & 1, abort, st))) {
@@ -218,53 +227,71 @@ match_tc_kernel(Dims dims, const BlockDesc* __restrict__ blocks, const int4* __r
         }
         if (!ok) continue;
         tc_fence_after();
-        const int width = min(kChunkCols, ndst_pad - c * kChunkCols);
-        const int hw = width >> 1;                       // multiple of 32
-        const int col0 = c * kChunkCols + half * hw;
-        for (int g = 0; g < hw; g += 32) {
-          uint32_t r[32];
-          tmem_ld32(tmem + lane_off + bb * kChunkCols + half * hw + g, r);
-          tmem_wait_ld();
-          const int cb = col0 + g;
-          const float4* invp = reinterpret_cast<const float4*>(sm.inv_d + cb);
+        const int width = min(kChunkCols, ndst_pad - c * kChunkCols);   // multiple of 64
+        auto scan = [&](const uint32_t (&r)[32], int cb) {
           if (cb + 32 <= ndst) {
+            const float4* invp = reinterpret_cast<const float4*>(sm.inv_d + cb);
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
               const float4 iv = invp[q];
               const float v0 = __uint_as_float(r[4 * q]) * iv.x, v1 = __uint_as_float(r[4 * q + 1]) * iv.y;
               const float v2 = __uint_as_float(r[4 * q + 2]) * iv.z, v3 = __uint_as_float(r[4 * q + 3]) * iv.w;
-              if (v0 > best) { best = v0; bi = cb + 4 * q; }
-              if (v1 > best) { best = v1; bi = cb + 4 * q + 1; }
-              if (v2 > best) { best = v2; bi = cb + 4 * q + 2; }
-              if (v3 > best) { best = v3; bi = cb + 4 * q + 3; }
+              if (v0 > bv[0]) { bv[0] = v0; bx[0] = cb + 4 * q; }
+              if (v1 > bv[1]) { bv[1] = v1; bx[1] = cb + 4 * q + 1; }
+              if (v2 > bv[2]) { bv[2] = v2; bx[2] = cb + 4 * q + 2; }
+              if (v3 > bv[3]) { bv[3] = v3; bx[3] = cb + 4 * q + 3; }
             }
           } else {
 #pragma unroll
             for (int q = 0; q < 32; ++q) {
               if (cb + q < ndst) {
                 const float v = __uint_as_float(r[q]) * sm.inv_d[cb + q];
-                if (v > best) { best = v; bi = cb + q; }
+                if (v > bv[q & 3]) { bv[q & 3] = v; bx[q & 3] = cb + q; }
               }
             }
           }
+        };
+        // this warp's groups: columns [32 g, 32 g + 32) for g = part, part + kParts (chunks of <= 256)
+        const int g0 = part * 32, g1 = (part + kParts) * 32;
+        uint32_t r0[32];
+        if (g0 < width) {
+          tmem_ld32(tmem + lane_off + bb * kChunkCols + g0, r0);
+          tmem_wait_ld();
+          scan(r0, c * kChunkCols + g0);
+        }
+        if (g1 < width) {
+          tmem_ld32(tmem + lane_off + bb * kChunkCols + g1, r0);
+          tmem_wait_ld();
+          scan(r0, c * kChunkCols + g1);
         }
         tc_fence_before();
         mbar_arrive(&sm.empty[bb]);
       }
-      sm.best_v[half][row] = best;
-      sm.best_i[half][row] = bi;
+      float best = bv[0];
+      int bi = bx[0];
+#pragma unroll
+      for (int j = 1; j < 4; ++j)
+        if (bv[j] > best || (bv[j] == best && bx[j] < bi)) {
+          best = bv[j];
+          bi = bx[j];
+        }
+      sm.best_v[part][row] = best;
+      sm.best_i[part][row] = bi;
       epi_sync();
-      if (half == 0 && ok) {
+      if (part == 0 && ok) {
         const int k = t * kRowsTile + row;
         if (k < nsrc) {
-          // the two column halves of one row: larger value, lower index on ties
+          // the column parts of one row: larger value, lower index on ties
           float v = sm.best_v[0][row];
           int i = sm.best_i[0][row];
-          const float v1 = sm.best_v[1][row];
-          const int i1 = sm.best_i[1][row];
-          if (v1 > v || (v1 == v && i1 < i)) {
-            v = v1;
-            i = i1;
+#pragma unroll
+          for (int p = 1; p < kParts; ++p) {
+            const float v1 = sm.best_v[p][row];
+            const int i1 = sm.best_i[p][row];
+            if (v1 > v || (v1 == v && i1 < i)) {
+              v = v1;
+              i = i1;
+            }
           }
           best_out[src0 + k] = i;
           score_out[src0 + k] = v * inv_s;

@@ -214,12 +214,14 @@ __global__ void __launch_bounds__(1024) out_scan_kernel(Dims dims, Buffers buf) 
   if (tid == 0) buf.state->n_items = (uint32_t)(dims.h * tq + tile_off[dims.h]);
 }
 
-// Per chunk: decide each query, write M_o, give outliers their slots and
-// copy each outlier's own row into its slot of Q~.
+// Per chunk: decide each query, write M_o, give outliers their ranks (the
+// slots after the head's regular ones) and copy each outlier's own row into
+// its slot of Q~.
 template <class T, int D>
 __global__ void __launch_bounds__(1024)
 out_emit_kernel(Dims dims, const T* __restrict__ Q, Buffers buf, int mask_injected) {
   __shared__ uint32_t tmp[40];
+  __shared__ int32_t list[kChunk];                     // this chunk's outliers in rank order
   constexpr int PER = kChunk / 1024;
   if (cta_plan_failed(buf.state)) return;
   const int c = blockIdx.x;
@@ -263,8 +265,7 @@ out_emit_kernel(Dims dims, const T* __restrict__ Q, Buffers buf, int mask_inject
     nout += out[j];
   }
   uint32_t rank = obefore + block_excl_scan(nout, tmp, &tot);
-  const T* Qh = Q + base * D;
-  T* Qt = reinterpret_cast<T*>(buf.q_tilde);
+  const uint32_t cnt = tot;                            // outliers of this chunk, ranks obefore + [0, cnt)
 #pragma unroll
   for (int j = 0; j < PER; ++j) {
     const int n = n0 + j;
@@ -273,14 +274,20 @@ out_emit_kernel(Dims dims, const T* __restrict__ Q, Buffers buf, int mask_inject
     if (out[j]) {
       buf.q_orank[base + n] = (int32_t)rank;
       buf.o_tok[(size_t)buf.out_base[hh] + rank - dims.out_base] = n;
-      const T* src = Qh + (size_t)n * D;
-      T* dst = Qt + ((size_t)buf.out_base[hh] + rank) * D;
-      constexpr int VEC = (int)(D * sizeof(T) / 16);
-#pragma unroll
-      for (int v = 0; v < VEC; ++v)
-        reinterpret_cast<uint4*>(dst)[v] = __ldg(reinterpret_cast<const uint4*>(src) + v);
+      list[rank - obefore] = n;
       ++rank;
     }
+  }
+  __syncthreads();
+  // each outlier's own row into its slot of Q~, 16-byte vectors spread over
+  // the threads (consecutive threads: consecutive parts of one row, then of
+  // the next outlier's row)
+  constexpr int VEC = (int)(D * sizeof(T) / 16);
+  const uint4* Qh = reinterpret_cast<const uint4*>(Q + base * D);
+  uint4* Qt = reinterpret_cast<uint4*>(reinterpret_cast<T*>(buf.q_tilde) + ((size_t)buf.out_base[hh] + obefore) * D);
+  for (uint32_t e = threadIdx.x; e < cnt * VEC; e += blockDim.x) {
+    const uint32_t i = e / VEC, v = e - i * VEC;
+    Qt[e] = __ldg(Qh + (size_t)list[i] * VEC + v);
   }
 }
 
