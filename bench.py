@@ -332,20 +332,60 @@ def roofline_of(w, r, steps: int):
     es = 4 if w.fp32 else 2
     row = w.d * es
     hn = w.h * w.N
-    mem_bytes = {
-        # read Q, K, V; write Q~ (regular slots), K~, V~; per-token slot and deviation key
-        "merge": 3 * hn * row + (w.h * plan.info.q_slots + 2 * w.h * plan.info.kv_slots) * row + 8 * hn,
-        # read O~ once, write out in original order, read the slot map
-        "unmerge": hn * row + r["sum_lq"] * row + 4 * hn,
-    }
+    sum_lq = r["sum_lq"]
+    n_out = sum_lq - w.h * plan.info.q_slots
+    kv_rows = w.h * plan.info.kv_slots
     hbm = pk["hbm_gbs"]
-    mem = {}
-    for k, b in mem_bytes.items():
-        ms = r["stages"][k][0] / steps
-        if ms > 0:
-            mem[k] = {"algorithmic_bytes": b, "ms": round(ms, 4), "GBps": round(b / ms / 1e6, 1),
-                      "frac_of_measured_hbm": round(b / ms / 1e6 / hbm, 4)}
-    return roof, mem
+
+    def per_ms(b, ms):
+        return {"algorithmic_bytes": int(b), "ms": round(ms, 4), "GBps": round(b / ms / 1e6, 1),
+                "frac_of_measured_hbm": round(b / ms / 1e6 / hbm, 4), "frac_of_8TBps": round(b / ms / 8e9, 4)}
+
+    st = {k: v[0] / steps for k, v in r["stages"].items()}
+    # the memory stages as one row: top-r merge, outlier filter and restore,
+    # unmerge.  Bytes the method must move: read Q, K, V; re-read the
+    # outliers' rows; write Q~ (regular and outlier rows), K~, V~; slot maps
+    # and deviations (~20 B per token and head); read O~ and write out.
+    total = (3 * hn * row + n_out * row + (sum_lq + 2 * kv_rows) * row + 20 * hn + sum_lq * row + hn * row)
+    mem = {"merge+outlier+unmerge": per_ms(total, st["merge"] + st["outlier"] + st["unmerge"])}
+    # per stage: merge reads Q, K, V and writes Q~ regular rows, K~, V~, the
+    # slot map and the deviation keys; unmerge reads O~ and the slot map and
+    # writes out
+    parts = {"merge": 3 * hn * row + (w.h * plan.info.q_slots + 2 * kv_rows) * row + 8 * hn,
+             "unmerge": hn * row + sum_lq * row + 4 * hn}
+    for k, b in parts.items():
+        if st[k] > 0:
+            mem[k] = per_ms(b, st[k])
+    # matching: 2 * n_dst * d flops per source on the tensor cores, and one
+    # argmax element per (source, destination) pair on the CUDA cores
+    pairs = 0
+    for stride in (w.q_stride, w.kv_stride):
+        for nb in block_sizes(w):
+            nd = -(-nb // stride)
+            pairs += (nb - nd) * nd
+    pairs *= w.h
+    mflops = 2.0 * pairs * w.d
+    match = None
+    if st["match"] > 0:
+        tf = mflops / (st["match"] / 1e3) / 1e12
+        match = {"ms": round(st["match"], 4), "algorithmic_flops": mflops, "TFLOPs": round(tf, 2),
+                 "frac_of_tensor_sustained": round(tf / peak, 4), "argmax_elements": pairs,
+                 "argmax_G_per_s": round(pairs / (st["match"] / 1e3) / 1e9, 1)}
+    return roof, mem, match
+
+
+def block_sizes(w):
+    """Token counts of the merge blocks of one head (HTTM note, key design 2:
+    n_s patches of n_t frames; contiguous runs in the contiguous variant)."""
+    from token_merging_view_b200.workloads import CONTIGUOUS
+    if w.mode == CONTIGUOUS:
+        return [min(w.contig_block, w.N - s) for s in range(0, w.N, w.contig_block)]
+    out = []
+    for t0 in range(0, w.T, w.n_t):
+        tg = min(w.n_t, w.T - t0)
+        for p0 in range(0, w.P, w.n_s):
+            out.append(tg * min(w.n_s, w.P - p0))
+    return out
 
 
 def run_ours(args):
@@ -365,7 +405,7 @@ def run_ours(args):
     r = measure_layer(w, args.steps, args.warmup, rank, world, dev)
     ms_step = r["ms_step"]
     value = world * w.N / (ms_step / 1e3)
-    roof, mem = roofline_of(w, r, args.steps)
+    roof, mem, match = roofline_of(w, r, args.steps)
     Q = r["Q"]
     es = 4 if w.fp32 else 2
 
@@ -406,10 +446,10 @@ def run_ours(args):
     if not args.no_secondary and world == 1 and args.workload != "vggt_500f":
         w2 = WORKLOADS["vggt_500f"]
         r2 = measure_layer(w2, 3, 2, rank, world, dev, with_e2e=False)
-        roof2, mem2 = roofline_of(w2, r2, 3)
+        roof2, mem2, match2 = roofline_of(w2, r2, 3)
         secondary = {"workload": w2.name, "tokens": w2.N, "value": round(w2.N / (r2["ms_step"] / 1e3), 1),
                      "unit": "tokens/s", "ms_per_step": round(r2["ms_step"], 3), "steps": 3,
-                     "roofline": roof2, "memory_stages": mem2,
+                     "roofline": roof2, "memory_stages": mem2, "match": match2,
                      "stage_ms_per_step": {k: round(v[0] / 3, 4) for k, v in r2["stages"].items()}}
         del r2
         torch.cuda.empty_cache()
@@ -438,6 +478,7 @@ def run_ours(args):
             "gpu_launches": launches,
             "roofline": roof,
             "memory_stages": mem,
+            "match": match,
             "stage_ms_per_step": {k: round(v[0] / args.steps, 4) for k, v in stages.items()},
             "dense_attention_same_length": dense,
             "cached_merge_indices": cached,
