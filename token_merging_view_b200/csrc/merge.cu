@@ -18,6 +18,7 @@
 
 #include "common.cuh"
 #include "launch.h"
+#include "tc_ptx.cuh"
 
 namespace httm {
 namespace {
@@ -77,22 +78,34 @@ struct Chunk {
       v[2] = __uint_as_float(w.z); v[3] = __uint_as_float(w.w);
     }
   }
+  // acc += row, element by element (pairs of fp32 lanes per instruction:
+  // the same sums as one add per element)
   __device__ static void add(float (&acc)[EPC], const uint4& w) {
     float v[EPC];
     unpack(w, v);
 #pragma unroll
-    for (int e = 0; e < EPC; ++e) acc[e] += v[e];
+    for (int e = 0; e < EPC; e += 2) {
+      float a0, a1;
+      tc::f2_unpack(tc::f2_add(tc::f2_pack(acc[e], acc[e + 1]), tc::f2_pack(v[e], v[e + 1])), a0, a1);
+      acc[e] = a0;
+      acc[e + 1] = a1;
+    }
   }
+  // sum over the chunk of (row - mean)^2: even and odd elements in two
+  // fp32 lanes, added at the end
   __device__ static float sq_dist(const uint4& w, const float (&mean)[EPC]) {
     float v[EPC];
     unpack(w, v);
-    float ss = 0.f;
+    const unsigned long long m1 = tc::f2_pack(-1.f, -1.f);
+    unsigned long long ss = 0ull;                      // (0.f, 0.f)
 #pragma unroll
-    for (int e = 0; e < EPC; ++e) {
-      const float d = v[e] - mean[e];
-      ss = fmaf(d, d, ss);
+    for (int e = 0; e < EPC; e += 2) {
+      const unsigned long long d = tc::f2_fma(tc::f2_pack(mean[e], mean[e + 1]), m1, tc::f2_pack(v[e], v[e + 1]));
+      ss = tc::f2_fma(d, d, ss);
     }
-    return ss;
+    float s0, s1;
+    tc::f2_unpack(ss, s0, s1);
+    return s0 + s1;
   }
   // Sum over the RPI lanes holding the same chunk of different rows; every
   // lane gets the same bits (the butterfly is symmetric).
