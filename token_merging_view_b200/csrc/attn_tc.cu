@@ -37,8 +37,9 @@
 // 16 log2 units above that max; P stays below 2^16 and most tiles never touch
 // O_t nor compute a max.  Sums use split accumulators for instruction-level
 // parallelism.  Every wait is bounded
-// (2 s): a wait that runs out sets HTTM_DEV_TIMEOUT, the CTA drains its MMAs,
-// frees TMEM and exits.
+// (WaitClock: 2 s of global time and 1 s of cycles at the top clock): a wait
+// that runs out sets HTTM_DEV_TIMEOUT, the CTA drains its MMAs, frees TMEM
+// and exits.
 #include <mutex>
 
 #include "common.cuh"
@@ -74,9 +75,9 @@ static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 
 // Bounded wait that ignores the abort flag (used to drain in-flight MMAs).
 __device__ bool drain_wait(uint64_t* bar, uint32_t parity) {
-  const unsigned long long t0 = globaltimer();
+  const WaitClock clk;
   while (!mbar_try_wait(bar, parity))
-    if (globaltimer() - t0 > kWaitTimeoutNs) return false;
+    if (clk.expired()) return false;
   return true;
 }
 

@@ -51,6 +51,10 @@ struct DevState {
   uint32_t n_items;              // live attention work items
   uint32_t plan_stamp;           // plan_id of the member lists held (0: none)
   uint32_t sel[8];               // outlier select: threshold key, eq budget, total
+  uint32_t wait_site;            // first bounded wait that ran out: barrier offset | parity << 20 | 1 << 31
+  uint32_t wait_cta;             // ... its CTA index
+  uint32_t wait_grid;            // ... and the grid size of its launch (tells the kernels apart)
+  uint32_t pad_;
 };
 
 struct Workspace {

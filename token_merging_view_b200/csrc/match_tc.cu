@@ -67,9 +67,9 @@ __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_gr
 __device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory"); }
 
 __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
-  const unsigned long long t0 = globaltimer();
+  const WaitClock clk;
   while (!mbar_try_wait(bar, parity))
-    if (globaltimer() - t0 > kWaitTimeoutNs) return false;
+    if (clk.expired()) return false;
   return true;
 }
 
@@ -303,7 +303,7 @@ match_tc_kernel(Dims dims, const BlockDesc* __restrict__ blocks, const int4* __r
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == kEpiThreads / 32) {          // the warp that allocated
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

@@ -799,6 +799,9 @@ __global__ void zero_state_kernel(Buffers buf, int keep_stamp) {
     buf.state->status = 0u;
     buf.state->n_eligible = 0u;
     buf.state->n_items = 0u;
+    buf.state->wait_site = 0u;
+    buf.state->wait_cta = 0u;
+    buf.state->wait_grid = 0u;
   }
   if (threadIdx.x < 8) buf.state->sel[threadIdx.x] = 0u;
 }

@@ -24,6 +24,7 @@ namespace httm {
 namespace tc {
 
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s for any single wait inside a CTA
+constexpr unsigned long long kWaitTimeoutCycles = 2000000000ull;  // ~1 s at the 1965 MHz top SM clock
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -34,6 +35,27 @@ __device__ __forceinline__ unsigned long long globaltimer() {
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
+
+__device__ __forceinline__ unsigned long long sm_cycles() {
+  unsigned long long c;
+  asm volatile("mov.u64 %0, %%clock64;" : "=l"(c));
+  return c;
+}
+
+// A bounded wait's clock: the nanosecond global timer together with this
+// SM's cycle counter.  The global timer is kept in step with the host clock
+// by the driver and may move forward in a jump; the cycle counter cannot
+// jump but runs slower at low clocks.  A wait ends only when both say it has
+// gone on too long (>= kWaitTimeoutNs of global time and >= 1 s worth of
+// cycles at the top SM clock), so it stays bounded (a few seconds at most)
+// and a timer jump alone does not end it.
+struct WaitClock {
+  unsigned long long ns0, cyc0;
+  __device__ __forceinline__ WaitClock() : ns0(globaltimer()), cyc0(sm_cycles()) {}
+  __device__ __forceinline__ bool expired() const {
+    return globaltimer() - ns0 > kWaitTimeoutNs && sm_cycles() - cyc0 > kWaitTimeoutCycles;
+  }
+};
 
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
@@ -62,18 +84,41 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Waits for the phase of `parity` to complete.  Gives up after
-// kWaitTimeoutNs or when *abort is set: then it sets *abort and the
+// Non-blocking: has the phase of `parity` completed?
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// A bounded wait on `bar` ran out: the first such wait records where it was
+// (barrier offset, parity, CTA, grid size), and HTTM_DEV_TIMEOUT is set.
+__device__ __forceinline__ void record_timeout(DevState* st, uint64_t* bar, uint32_t parity) {
+  if (atomicCAS(&st->wait_site, 0u, 0x80000000u | (parity & 1u) << 20 | (smem_u32(bar) & 0xFFFFFu)) == 0u) {
+    st->wait_cta = blockIdx.x;
+    st->wait_grid = gridDim.x;
+  }
+  set_status(st, HTTM_DEV_TIMEOUT);
+}
+
+// Waits for the phase of `parity` to complete.  Gives up when its WaitClock
+// expires or when *abort is set: then it sets *abort and the
 // HTTM_DEV_TIMEOUT status bit and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, DevState* st) {
   if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = globaltimer();
+  const WaitClock clk;
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (globaltimer() - t0 > kWaitTimeoutNs) {
+    if (clk.expired()) {
       *abort = 1;
-      set_status(st, HTTM_DEV_TIMEOUT);
+      record_timeout(st, bar, parity);
       return false;
     }
   }
