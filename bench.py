@@ -7,8 +7,9 @@ own independent layer (weak scaling, no data-path collective).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload vggt_100f]
     python bench.py --impl reference ...   # the fp64 CPU oracle on a bounded sample
+    python bench.py --sweep                # 1000-frame sweep of merge / outlier ratios and plan variants
 
-Prints one JSON line (rank 0).
+Prints one JSON line (rank 0); --sweep prints one line per sweep point.
 """
 from __future__ import annotations
 
@@ -38,6 +39,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-secondary", action="store_true", help="skip the 500-frame layer")
+    ap.add_argument("--sweep", action="store_true",
+                    help="1000-frame sweep: Q r x outlier d x (head-wise temporal, head-uniform, contiguous)")
+    ap.add_argument("--sweep-rows", type=int, default=128, help="sampled query rows per head for the output error")
     return ap.parse_args()
 
 
@@ -491,6 +495,134 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+# ----------------------------------------------------------------------------
+# 1000-frame sweep of the merge settings and the plan variants
+# ----------------------------------------------------------------------------
+
+def sweep_points(w):
+    """Q merge ratio r x outlier ratio d (K/V r = 50 %), each with the three
+    plans: head-wise temporal blocks (HTTM), one head-uniform plan per block
+    (the mean over heads of the cosines, as ToMe/FastVGGT merge), and
+    contiguous un-reordered blocks of 3840 tokens (HTTM note, background
+    section and key design 2).  r = 85 % needs destinations every 8th token:
+    every 4th leaves only 75 % of a block as sources."""
+    from token_merging_view_b200.workloads import CONTIGUOUS, HEAD_UNIFORM, HEADWISE_TEMPORAL
+    pts = []
+    for r in (50, 70, 85):
+        for d in (0, 5, 10):
+            for mode, name in ((HEADWISE_TEMPORAL, "headwise_temporal"), (HEAD_UNIFORM, "head_uniform"),
+                               (CONTIGUOUS, "contiguous_3840")):
+                pts.append((name, w.with_(q_pct=r, q_stride=8 if r == 85 else 4, kv_pct=50, kv_stride=4,
+                                          out_pct=d, mode=mode, contig_block=3840)))
+    return pts
+
+
+def dense_rows(Q, K, V, idx, scale):
+    """softmax(q K^T * scale) V for the sampled query rows of every head, in
+    float64 on the device (torch), as the unmerged layer's reference."""
+    import torch
+    outs = []
+    for hh in range(Q.shape[0]):
+        q = Q[hh, idx[hh]].double()
+        s = (q @ K[hh].double().T) * scale
+        p = torch.softmax(s, dim=-1)
+        outs.append(p @ V[hh].double())
+        del s, p
+    return torch.stack(outs)
+
+
+def deviation_stats(Q, dbg, n_q_slots):
+    """Pre-filter query deviation ||q_n - q~_G(n)|| (mean, p99 over all h x N
+    tokens, 0 for singletons) and the deviation of each non-outlier from its
+    restored slot (mean over all non-outliers, and over those whose restored
+    slot still holds >= 2 tokens)."""
+    import torch
+    dev = dbg["dev"]
+    flat = dev.flatten()
+    k = max(1, int(0.99 * flat.numel()))
+    p99 = float(flat.kthvalue(k).values)
+    post_sum, post_n, post_m_sum, post_m_n = 0.0, 0, 0.0, 0
+    for hh in range(Q.shape[0]):
+        slot = dbg["q_slot"][hh].long()
+        # outliers own slots past the regular ones: never index with those
+        keep = (dbg["outlier"][hh] == 0) & (slot >= 0) & (slot < n_q_slots)
+        s_reg = torch.where(keep, slot, torch.zeros_like(slot))
+        cnt = torch.bincount(s_reg[keep], minlength=n_q_slots)
+        merged = cnt[s_reg] >= 2
+        diff = Q[hh].float() - dbg["q_restored"][hh][s_reg]
+        dn = diff.norm(dim=-1)
+        post_sum += float(dn[keep].sum())
+        post_n += int(keep.sum())
+        sel = keep & merged
+        post_m_sum += float(dn[sel].sum())
+        post_m_n += int(sel.sum())
+    return {"pre_filter_dev_mean": round(float(flat.mean()), 5), "pre_filter_dev_p99": round(p99, 5),
+            "restored_dev_mean_non_outliers": round(post_sum / max(1, post_n), 5),
+            "restored_dev_mean_merged_non_outliers": round(post_m_sum / max(1, post_m_n), 5)}
+
+
+def run_sweep(args):
+    import torch
+
+    from token_merging_view_b200 import binding as B
+    from token_merging_view_b200.inputs import make_qkv
+    from token_merging_view_b200.workloads import WORKLOADS
+
+    rank, world, local = dist_env()
+    if rank != 0:
+        return
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = WORKLOADS["vggt_1000f"]
+    Q, K, V = make_qkv(T=w.T, grid=w.grid, h=w.h, d=w.d, seed=w.seed, noise_sigma=w.noise_sigma,
+                       max_shift=w.max_shift, dtype=torch.bfloat16, device=dev)
+    g = torch.Generator(device="cpu").manual_seed(1234)
+    idx = torch.stack([torch.randperm(w.N, generator=g)[: args.sweep_rows].sort().values for _ in range(w.h)]).to(dev)
+    scale = w.d ** -0.5
+    ref = dense_rows(Q, K, V, idx, scale)
+    out = torch.empty_like(Q)
+    stream = torch.cuda.current_stream()
+    base_rows = {}
+    for name, pw in sweep_points(w):
+        plan = B.httm_plan(B.LayerConfig.from_workload(pw))
+        ws = plan.new_workspace(dev)
+        dbg = B.debug_buffers(plan, dev)
+        B.httm_forward_debug(plan, Q, K, V, dbg, out=out, workspace=ws)     # also the warm-up
+        status = B.httm_get_device_status(plan, ws)
+        n_out = int(B.workspace_view(plan, ws, "n_out").sum())
+        stats = deviation_stats(Q, dbg, plan.info.q_slots)
+        rows = torch.stack([out[hh, idx[hh]] for hh in range(w.h)]).double()
+        err = (rows - ref).norm() / ref.norm()
+        key = (pw.q_pct, pw.out_pct)
+        if name == "headwise_temporal":
+            base_rows[key] = rows
+        vs_ht = (rows - base_rows[key]).norm() / base_rows[key].norm() if key in base_rows else None
+        del dbg
+        steps = 2
+        plan.profile(True)
+        plan.profile_read()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            B.httm_forward(plan, Q, K, V, out=out, workspace=ws, stream=stream)
+        b.record(stream)
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / steps
+        stages = {k: round(v[0] / steps, 3) for k, v in plan.profile_read().items()}
+        line = {"sweep": w.name, "plan": name, "q_merge_pct": pw.q_pct, "q_dst_stride": pw.q_stride,
+                "kv_merge_pct": pw.kv_pct, "outlier_pct": pw.out_pct, "status": status,
+                "tokens_per_s": round(w.N / (ms / 1e3), 1), "ms_per_step": round(ms, 2), "steps": steps,
+                "q_rows": w.h * plan.info.q_slots + n_out, "kv_rows_per_head": plan.info.kv_slots,
+                "stage_ms": stages, **stats,
+                "out_rel_l2_vs_dense_sampled": round(float(err), 5),
+                "out_rel_l2_vs_headwise_temporal_sampled": None if vs_ht is None else round(float(vs_ht), 5),
+                "sampled_rows_per_head": args.sweep_rows}
+        print(json.dumps(line), flush=True)
+        del ws, plan
+        torch.cuda.empty_cache()
+
+
 def run_reference(args):
     rank, world, local = dist_env()
     if rank != 0:
@@ -527,6 +659,8 @@ def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+    elif args.sweep:
+        run_sweep(args)
     else:
         run_ours(args)
 
