@@ -8,6 +8,7 @@ own independent layer (weak scaling, no data-path collective).
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload vggt_100f]
     python bench.py --impl reference ...   # the fp64 CPU oracle on a bounded sample
     python bench.py --sweep                # 1000-frame sweep of merge / outlier ratios and plan variants
+    python bench.py --block-sweep          # block shapes n_s x n_t on the 100-frame layer
 
 Prints one JSON line (rank 0); --sweep prints one line per sweep point.
 """
@@ -42,6 +43,8 @@ def parse():
     ap.add_argument("--sweep", action="store_true",
                     help="1000-frame sweep: Q r x outlier d x (head-wise temporal, head-uniform, contiguous)")
     ap.add_argument("--sweep-rows", type=int, default=128, help="sampled query rows per head for the output error")
+    ap.add_argument("--block-sweep", action="store_true",
+                    help="100-frame layer: spatial (n_t = 1) against spatio-temporal block shapes at three block sizes")
     return ap.parse_args()
 
 
@@ -583,6 +586,7 @@ def run_sweep(args):
     out = torch.empty_like(Q)
     stream = torch.cuda.current_stream()
     base_rows = {}
+    clocks = Clocks(dev.index if dev.index is not None else 0)
     for name, pw in sweep_points(w):
         plan = B.httm_plan(B.LayerConfig.from_workload(pw))
         ws = plan.new_workspace(dev)
@@ -621,6 +625,82 @@ def run_sweep(args):
         print(json.dumps(line), flush=True)
         del ws, plan
         torch.cuda.empty_cache()
+    print(json.dumps({"sweep": w.name, "clocks": clocks.stop()}), flush=True)
+
+
+def block_shapes():
+    """(n_s, n_t) pairs at three block sizes: a purely spatial block (n_t = 1,
+    n_s <= 1369 patches of one frame) against the same number of tokens
+    spread over more frames (HTTM note, key design 2 and the spatial /
+    temporal trade-off of its analysis section)."""
+    return {
+        "~800": [(800, 1), (400, 2), (200, 4), (100, 8), (50, 16), (27, 30)],
+        "~1369": [(1369, 1), (685, 2), (343, 4), (172, 8), (92, 15), (46, 30)],
+        "~3840": [(1280, 3), (640, 6), (384, 10), (256, 15), (128, 30), (64, 60)],
+    }
+
+
+def run_block_sweep(args):
+    import torch
+
+    from token_merging_view_b200 import binding as B
+    from token_merging_view_b200.inputs import make_qkv
+    from token_merging_view_b200.workloads import WORKLOADS
+
+    rank, world, local = dist_env()
+    if rank != 0:
+        return
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = WORKLOADS["vggt_100f"]
+    Q, K, V = make_qkv(T=w.T, grid=w.grid, h=w.h, d=w.d, seed=w.seed, noise_sigma=w.noise_sigma,
+                       max_shift=w.max_shift, dtype=torch.bfloat16, device=dev)
+    out = torch.empty_like(Q)
+    stream = torch.cuda.current_stream()
+    clocks = Clocks(dev.index if dev.index is not None else 0)
+    for size, shapes in block_shapes().items():
+        for n_s, n_t in shapes:
+            pw = w.with_(n_s=n_s, n_t=n_t)
+            plan = B.httm_plan(B.LayerConfig.from_workload(pw))
+            ws = plan.new_workspace(dev)
+            dbg = B.debug_buffers(plan, dev)
+            B.httm_forward_debug(plan, Q, K, V, dbg, out=out, workspace=ws)     # also the warm-up
+            status = B.httm_get_device_status(plan, ws)
+            stats = deviation_stats(Q, dbg, plan.info.q_slots)
+            kdev = None
+            if dbg.get("k_means") is not None:
+                # key deviation from the key means, per token (0 for singletons)
+                ks, tot, n = dbg["k_slot"], 0.0, 0
+                for hh in range(w.h):
+                    sl = ks[hh].long()
+                    d = (K[hh].float() - dbg["k_means"][hh][sl]).norm(dim=-1)
+                    tot += float(d.sum())
+                    n += d.numel()
+                kdev = round(tot / max(1, n), 5)
+            del dbg
+            steps = 5
+            plan.profile(True)
+            plan.profile_read()
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(steps):
+                B.httm_forward(plan, Q, K, V, out=out, workspace=ws, stream=stream)
+            b.record(stream)
+            torch.cuda.synchronize()
+            ms = a.elapsed_time(b) / steps
+            stages = {k: round(v[0] / steps, 4) for k, v in plan.profile_read().items()}
+            line = {"block_sweep": w.name, "block_size": size, "n_s": n_s, "n_t": n_t,
+                    "n_b_full": n_s * n_t, "blocks_per_head": plan.info.n_blocks, "status": status,
+                    "tokens_per_s": round(w.N / (ms / 1e3), 1), "ms_per_step": round(ms, 3), "stage_ms": stages,
+                    "q_pre_filter_dev_mean": stats["pre_filter_dev_mean"],
+                    "q_pre_filter_dev_p99": stats["pre_filter_dev_p99"],
+                    "q_restored_dev_mean_non_outliers": stats["restored_dev_mean_non_outliers"],
+                    "k_dev_mean": kdev}
+            print(json.dumps(line), flush=True)
+            del ws, plan
+            torch.cuda.empty_cache()
+    print(json.dumps({"block_sweep": w.name, "clocks": clocks.stop()}), flush=True)
 
 
 def run_reference(args):
@@ -661,6 +741,8 @@ def main():
         run_reference(args)
     elif args.sweep:
         run_sweep(args)
+    elif args.block_sweep:
+        run_block_sweep(args)
     else:
         run_ours(args)
 
