@@ -120,6 +120,7 @@ Workspace layout(const Dims& d, bool fp32) {
   w.k_tilde = take((size_t)d.h * d.k_slots * d.d * es);
   w.v_tilde = take((size_t)d.h * d.k_slots * d.d * es);
   w.o_tilde = take((size_t)d.q_rows_alloc * d.d * es);
+  w.attn_part = take((size_t)kMaxAttnParts * kAttnRows * kAttnPartStride * 4);
   w.total = off;
   return w;
 }
@@ -154,6 +155,7 @@ Buffers resolve(const Workspace& w, void* base) {
   b.k_tilde = p + w.k_tilde;
   b.v_tilde = p + w.v_tilde;
   b.o_tilde = p + w.o_tilde;
+  b.attn_part = reinterpret_cast<float*>(p + w.attn_part);
   return b;
 }
 
@@ -201,11 +203,19 @@ httm_status check_device(httm_plan_s* plan) {
     if (e_ != cudaSuccess) return HTTM_ERR_CUDA;      \
   } while (0)
 
+// The attention stage: the tensor-core kernel plus the merge of the last
+// wave's split items (two launches, timed as one stage), or the CUDA-core
+// kernel.  Adds its launches to *launches.
 httm_status attention(const httm_plan_s* plan, const void* q, const void* k, const void* v, void* o, int Lk,
-                      const Buffers& buf, cudaStream_t s) {
+                      const Buffers& buf, cudaStream_t s, int* launches) {
   cudaError_t e;
-  if (attention_tc_supported(plan->dims, plan->fp32)) e = launch_attention_tc(plan->dims, q, k, v, o, Lk, buf, s);
-  else e = launch_attention_simt(plan->dims, plan->fp32, q, k, v, o, Lk, buf, s);
+  if (attention_tc_supported(plan->dims, plan->fp32)) {
+    e = launch_attention_tc(plan->dims, q, k, v, o, Lk, buf, s);
+    *launches += 2;
+  } else {
+    e = launch_attention_simt(plan->dims, plan->fp32, q, k, v, o, Lk, buf, s);
+    *launches += 1;
+  }
   return e == cudaSuccess ? HTTM_OK : HTTM_ERR_CUDA;
 }
 
@@ -243,8 +253,7 @@ httm_status forward_impl(httm_plan_s* plan, const void* Q, const void* K, const 
   }
   if (dims.mode == HTTM_DENSE) {
     StageTimer t(plan, s, HTTM_STAGE_ATTENTION, 1);
-    st = attention(plan, Q, K, V, out, dims.N, buf, s);
-    ++launches;
+    st = attention(plan, Q, K, V, out, dims.N, buf, s, &launches);
     plan->launches = launches;
     return st;
   }
@@ -278,8 +287,7 @@ httm_status forward_impl(httm_plan_s* plan, const void* Q, const void* K, const 
   }
   {
     StageTimer t(plan, s, HTTM_STAGE_ATTENTION, 1);
-    st = attention(plan, buf.q_tilde, buf.k_tilde, buf.v_tilde, buf.o_tilde, dims.k_slots, buf, s);
-    ++launches;
+    st = attention(plan, buf.q_tilde, buf.k_tilde, buf.v_tilde, buf.o_tilde, dims.k_slots, buf, s, &launches);
     if (st != HTTM_OK) return st;
   }
   {

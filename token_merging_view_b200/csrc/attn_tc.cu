@@ -26,8 +26,8 @@
 // buffer once S is in registers -- then O_0 [384, 448) and O_1 [448, 512).
 // Tensor-core operations complete in issue order: S product i + 3 reuses a
 // buffer only after the PV that read P from it, and a softmax sees S for
-// (0, j+1) before it finishes (0, j).  A softmax that rescales O_t waits for
-// PV(t, j-1) first.  Two warpgroups keep two softmax warps per SM
+// (0, j+1) before it finishes (0, j).  A softmax arrives for step j only
+// once PV(t, j-1) has completed (and rescales O_t only then).  Two warpgroups keep two softmax warps per SM
 // sub-partition busy on the exp unit while the tensor core alternates
 // between the tiles.
 //
@@ -40,6 +40,7 @@
 // (WaitClock: 2 s of global time and 1 s of cycles at the top clock): a wait
 // that runs out sets HTTM_DEV_TIMEOUT, the CTA drains its MMAs, frees TMEM
 // and exits.
+#include <algorithm>
 #include <mutex>
 
 #include "common.cuh"
@@ -81,19 +82,47 @@ __device__ bool drain_wait(uint64_t* bar, uint32_t parity) {
   return true;
 }
 
+// The last, partial wave of work items is split along the keys: with n items
+// and S SMs, the r = n mod S items of the last wave each become p CTAs
+// (p = min(4, S / r, key tiles)) over consecutive key-tile ranges, so that
+// the wave fills more SMs; each part writes O (unnormalised, fp32), its row
+// sums and maxima to the partial area, and attn_combine_kernel merges them.
+struct SplitPlan {
+  int n_full, r, p;   // items [0, n_full) whole; items [n_full, n_full + r) in p parts
+};
+__device__ __forceinline__ SplitPlan split_plan(int n, int S, int n_kv) {
+  const int r = S > 0 ? n % S : 0;
+  int p = r > 0 ? min(4, S / r) : 1;
+  p = min(p, n_kv);
+  if (p <= 1) return SplitPlan{n, 0, 1};
+  return SplitPlan{n - r, r, p};
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                const __grid_constant__ CUtensorMap tv, __nv_bfloat16* __restrict__ O, int Lk, float scale_log2,
-               Buffers buf) {
-  if (blockIdx.x >= buf.state->n_items) return;
+               int n_sm, Buffers buf) {
+  const int n_kv_all = (Lk + kBN - 1) / kBN;
+  const SplitPlan sp = split_plan((int)buf.state->n_items, n_sm, n_kv_all);
+  const int n_cta = sp.n_full + sp.r * sp.p;
+  if ((int)blockIdx.x >= n_cta) return;
   if (cta_plan_failed(buf.state)) return;
+  // this CTA's item and key tiles [j0, j0 + n_kv); part >= 0 for a split item
+  int item = blockIdx.x, part = -1, j0 = 0, n_kv = n_kv_all;
+  if ((int)blockIdx.x >= sp.n_full) {
+    const int k = blockIdx.x - sp.n_full;
+    item = sp.n_full + k / sp.p;
+    part = k;                                        // index of the partial result
+    const int q = k % sp.p;
+    j0 = q * n_kv_all / sp.p;
+    n_kv = (q + 1) * n_kv_all / sp.p - j0;
+  }
   extern __shared__ uint8_t smem_raw[];
   AttnSmem& sm = *reinterpret_cast<AttnSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int4 it = buf.items[blockIdx.x];
+  const int4 it = buf.items[item];
   const int hh = it.x, q_row0 = it.y, n_rows = it.z;
-  const int kv_row0 = hh * Lk;
-  const int n_kv = (Lk + kBN - 1) / kBN;
+  const int kv_row0 = hh * Lk + j0 * kBN;            // first key row of this CTA's range
   DevState* st = buf.state;
 
   if (threadIdx.x == 0) {
@@ -208,7 +237,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
       for (int c = 0; c < 4; ++c)
         tmem_ld32(ts + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
       tmem_wait_ld();
-      const int valid = Lk - j * kBN;
+      const int valid = Lk - (j0 + j) * kBN;
       if (valid < kBN) {
 #pragma unroll
         for (int i = 0; i < kBN; ++i)
@@ -222,6 +251,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
       // redo the tile.  Otherwise P stays below 2^16 and O_t is untouched.
       const unsigned long long cc = f2_pack(scale_log2, scale_log2);
       const bool live_row = t * kBM + row < n_rows;
+      bool pv_done = j == 0;                              // PV(t, j-1) seen complete
       float rsum = 0.f;
       for (int pass = 0; pass < 2; ++pass) {
         const unsigned long long mm = f2_pack(-m_used, -m_used);
@@ -264,10 +294,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         const float m_new = fmaxf(m_used, mts);
         const float alpha = ex2(m_used - m_new);
         if (j > 0) {
-          if (!__all_sync(0xffffffffu, mbar_wait(&sm.o_done[t], (j - 1) & 1, abort, st))) {
+          if (!pv_done && !__all_sync(0xffffffffu, mbar_wait(&sm.o_done[t], (j - 1) & 1, abort, st))) {
             ok = false;
             break;
           }
+          pv_done = true;
           tc_fence_after();
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
@@ -284,11 +315,43 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
       }
       if (!ok) break;
       l += rsum;
+      // No arrival for step j before PV(t, j-1) has completed.  Parity waits
+      // are exact only while a barrier is at most one phase from the one
+      // awaited: this keeps o_done within one phase of every later wait on
+      // it (the rescale's, the next step's, the final one -- a two-tile item
+      // could otherwise see "phase 1 done" before PV(t, 0) finished), and
+      // since PV(t, j-1) follows the close of p_full's phase j-1, no warp can
+      // arrive for step j while a slower warp of its warpgroup has not yet
+      // arrived for step j-1 (p_full counts arrivals, not steps).
+      if (!pv_done && !__all_sync(0xffffffffu, mbar_wait(&sm.o_done[t], (j - 1) & 1, abort, st))) {
+        ok = false;
+        break;
+      }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&sm.p_full[t]);
     }
-    if (ok && __all_sync(0xffffffffu, mbar_wait(&sm.o_done[t], (n_kv - 1) & 1, abort, st))) {
+    const bool done = ok && __all_sync(0xffffffffu, mbar_wait(&sm.o_done[t], (n_kv - 1) & 1, abort, st));
+    if (done && part >= 0) {
+      // a part of a split item: O unnormalised, the row sum and the max in
+      // use, for attn_combine_kernel
+      tc_fence_after();
+      const int r = t * kBM + row;
+      float* dst = buf.attn_part + ((size_t)part * kAttnRows + r) * kAttnPartStride;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t o[32];
+        tmem_ld32(to + c * 32, o);
+        tmem_wait_ld();
+#pragma unroll
+        for (int v = 0; v < 8; ++v)
+          reinterpret_cast<float4*>(dst)[c * 8 + v] =
+              make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]), __uint_as_float(o[4 * v + 2]),
+                          __uint_as_float(o[4 * v + 3]));
+      }
+      dst[kD] = l;
+      dst[kD + 1] = m_used;
+    } else if (done) {
       tc_fence_after();
       const float inv = 1.f / l;
       uint32_t packed[32];
@@ -320,6 +383,48 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
     }
     tc_fence_after();
     tmem_dealloc(tmem, 512);
+  }
+}
+
+// Merge the parts of each split item (see split_plan): with M the largest
+// max in use, O = sum_p O_p 2^(m_p - M) / sum_p l_p 2^(m_p - M), in part
+// order; rows past the item's end are left alone.
+__global__ void __launch_bounds__(kAttnRows)
+attn_combine_kernel(__nv_bfloat16* __restrict__ O, int Lk, int n_sm, Buffers buf) {
+  if (plan_failed(buf.state)) return;
+  const SplitPlan sp = split_plan((int)buf.state->n_items, n_sm, (Lk + kBN - 1) / kBN);
+  for (int i = blockIdx.x; i < sp.r; i += gridDim.x) {
+    const int4 it = buf.items[sp.n_full + i];
+    for (int r = threadIdx.x; r < it.z; r += blockDim.x) {
+      const float* src[4];
+      float w[4], mx = -INFINITY, l = 0.f;
+      for (int q = 0; q < sp.p; ++q) {
+        src[q] = buf.attn_part + ((size_t)(i * sp.p + q) * kAttnRows + r) * kAttnPartStride;
+        mx = fmaxf(mx, src[q][kD + 1]);
+      }
+      for (int q = 0; q < sp.p; ++q) {
+        w[q] = ex2(src[q][kD + 1] - mx);
+        l = fmaf(src[q][kD], w[q], l);
+      }
+      const float inv = 1.f / l;
+      uint4* dst = reinterpret_cast<uint4*>(O + ((size_t)it.y + r) * kD);
+#pragma unroll
+      for (int v = 0; v < 8; ++v) {
+        float a[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) a[e] = 0.f;
+        for (int q = 0; q < sp.p; ++q) {
+          const float4 x0 = reinterpret_cast<const float4*>(src[q])[2 * v];
+          const float4 x1 = reinterpret_cast<const float4*>(src[q])[2 * v + 1];
+          a[0] = fmaf(x0.x, w[q], a[0]); a[1] = fmaf(x0.y, w[q], a[1]);
+          a[2] = fmaf(x0.z, w[q], a[2]); a[3] = fmaf(x0.w, w[q], a[3]);
+          a[4] = fmaf(x1.x, w[q], a[4]); a[5] = fmaf(x1.y, w[q], a[5]);
+          a[6] = fmaf(x1.z, w[q], a[6]); a[7] = fmaf(x1.w, w[q], a[7]);
+        }
+        dst[v] = make_uint4(pack_bf16(a[0] * inv, a[1] * inv), pack_bf16(a[2] * inv, a[3] * inv),
+                            pack_bf16(a[4] * inv, a[5] * inv), pack_bf16(a[6] * inv, a[7] * inv));
+      }
+    }
   }
 }
 
@@ -372,8 +477,19 @@ cudaError_t launch_attention_tc(const Dims& dims, const void* q, const void* k, 
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   const float scale_log2 = dims.scale * 1.4426950408889634f;
-  attn_tc_kernel<<<dims.max_items, kThreads, kSmemBytes, s>>>(tq, tk, tv, static_cast<__nv_bfloat16*>(o), Lk,
-                                                              scale_log2, buf);
+  static int n_sm_cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidValue;
+  int& n_sm = n_sm_cached[dev & 63];
+  if (n_sm == 0 && cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return cudaErrorInvalidValue;
+  const int S = std::min(n_sm, kMaxAttnParts);
+  // up to S extra CTAs for the split parts of the last wave
+  attn_tc_kernel<<<dims.max_items + S, kThreads, kSmemBytes, s>>>(tq, tk, tv, static_cast<__nv_bfloat16*>(o), Lk,
+                                                                  scale_log2, S, buf);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  attn_combine_kernel<<<S, kAttnRows, 0, s>>>(static_cast<__nv_bfloat16*>(o), Lk, S, buf);
   return cudaGetLastError();
 }
 

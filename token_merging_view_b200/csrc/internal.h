@@ -43,6 +43,9 @@ struct Dims {
 constexpr int kChunk = 4096;       // keys per chunk of the outlier compaction
 constexpr int kHistBins = 2048;    // radix digit of the outlier select (11 bits)
 constexpr int kAttnRows = 256;     // query rows per attention work item (two 128-row tiles)
+constexpr int kMaxAttnParts = 256; // partial results of the last wave's split items (<= one per SM)
+constexpr int kAttnPartStride = 68; // floats per partial row: O (64), row sum, max in use, 2 unused (16-byte rows)
+static_assert(kAttnPartStride * 4 % 16 == 0, "partial rows are read and written as float4");
 
 // Device-side state at the head of the workspace.
 struct DevState {
@@ -62,6 +65,7 @@ struct Workspace {
   size_t q_best, q_score, q_merged, k_best, k_score, k_merged;
   size_t q_slot, q_orank, o_tok, keys, mask, q_members, q_gstart, q_gcount, k_members, k_gstart, k_gcount;
   size_t q_tilde, k_tilde, v_tilde, o_tilde;
+  size_t attn_part;
   size_t total;
 };
 
@@ -89,6 +93,7 @@ struct Buffers {
   int32_t* k_gstart;
   int32_t* k_gcount;
   void* q_tilde; void* k_tilde; void* v_tilde; void* o_tilde;
+  float* attn_part;        // [kMaxAttnParts][kAttnRows][kAttnPartStride]: partial attention of split items
 };
 
 }  // namespace httm
