@@ -212,3 +212,24 @@ def test_host_errors():
     with pytest.raises(B.HttmError) as e:
         B.httm_forward(plan, Qm, K, V, workspace=ws)
     assert e.value.status == 5
+
+
+@pytest.mark.parametrize("T", [1, 2])
+def test_short_key_ranges_split_parts(T):
+    """Few key tiles per head: every work item of the last (here the only)
+    wave runs as parts of one or two key tiles whose partial results are
+    merged.  Repeated calls must agree bit for bit, and with the oracle on
+    its own plan and mask (this case once exposed two barrier races)."""
+    w = MID.with_(T=T, n_t=T)
+    _, plan, cfg, (Q, K, V), (q, k, v) = _case(w)
+    res = O.forward_plan(cfg, q, k, v)
+    inj = PL.oracle_plan_tensors(res)
+    outs = []
+    for _ in range(4):
+        out, _, _, status = PL.run(plan, Q, K, V, injected=inj, debug=False)
+        assert status == 0
+        outs.append(out)
+    for o in outs[1:]:
+        assert torch.equal(o, outs[0])
+    mx, rl2 = PL.sample_out_error(res, PL.to64(outs[0]), cfg, 1 << 30)
+    assert mx <= PL.OUT_MAX_ABS and rl2 <= PL.OUT_REL_L2, (mx, rl2)
