@@ -268,45 +268,51 @@ def measure_layer(w, steps: int, warmup: int, rank: int, world: int, dev, with_e
     if with_e2e:
         # End to end through the same C ABI call, from pinned host memory:
         # every step copies its Q/K/V in and its output back.  Two device
-        # buffer sets and a copy stream pipeline the steps, as a caller of the
-        # asynchronous API would: step i+1's inputs travel while step i
-        # computes, and step i's output travels back behind it.
+        # buffer sets and one copy stream per direction pipeline the steps,
+        # as a caller of the asynchronous API would: step i+1's inputs travel
+        # in while step i computes and step i-1's output travels back (the
+        # link carries both directions at once).
         hQ, hK, hV = (t.cpu().pin_memory() for t in (Q, K, V))
         hO = [torch.empty(out.shape, dtype=out.dtype, pin_memory=True) for _ in range(2)]
         dIn = [(Q, K, V), tuple(torch.empty_like(t) for t in (Q, K, V))]
         dOut = [out, torch.empty_like(out)]
         ws2 = [ws, plan.new_workspace(dev)]
-        copy = torch.cuda.Stream(device=dev)
+        c_in = torch.cuda.Stream(device=dev)
+        c_out = torch.cuda.Stream(device=dev)
         ev_in = [torch.cuda.Event() for _ in range(2)]
         ev_done = [torch.cuda.Event() for _ in range(2)]
         ev_out = [torch.cuda.Event() for _ in range(2)]
         for e in ev_out:
-            e.record(copy)
+            e.record(c_out)
+        for e in ev_done:
+            e.record(stream)
 
         def e2e_run(n):
-            copy.wait_stream(stream)
-            with torch.cuda.stream(copy):
+            c_in.wait_stream(stream)
+            c_out.wait_stream(stream)
+            with torch.cuda.stream(c_in):
                 for t, h in zip(dIn[0], (hQ, hK, hV)):
                     t.copy_(h, non_blocking=True)
-                ev_in[0].record(copy)
+                ev_in[0].record(c_in)
             for i in range(n):
                 b = i & 1
                 if i + 1 < n:                   # prefetch the next step's inputs
                     nb = (i + 1) & 1
-                    with torch.cuda.stream(copy):
-                        copy.wait_event(ev_done[nb])
+                    with torch.cuda.stream(c_in):
+                        c_in.wait_event(ev_done[nb])
                         for t, h in zip(dIn[nb], (hQ, hK, hV)):
                             t.copy_(h, non_blocking=True)
-                        ev_in[nb].record(copy)
+                        ev_in[nb].record(c_in)
                 stream.wait_event(ev_in[b])
                 stream.wait_event(ev_out[b])    # the output buffer has been drained
                 B.httm_forward(plan, *dIn[b], out=dOut[b], workspace=ws2[b], stream=stream)
                 ev_done[b].record(stream)
-                with torch.cuda.stream(copy):
-                    copy.wait_event(ev_done[b])
+                with torch.cuda.stream(c_out):
+                    c_out.wait_event(ev_done[b])
                     hO[b].copy_(dOut[b], non_blocking=True)
-                    ev_out[b].record(copy)
-            stream.wait_stream(copy)
+                    ev_out[b].record(c_out)
+            stream.wait_stream(c_in)
+            stream.wait_stream(c_out)
 
         e2e_run(2)
         n = max(3, steps)

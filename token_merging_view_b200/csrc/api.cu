@@ -442,9 +442,11 @@ httm_status httm_plan(const httm_cfg* cfg, httm_plan_t* out) {
     p->items_h = std::move(items);
     // tensor-core matching: one CTA per (tensor, head, block), a block split in
     // runs of whole 128-source tiles when that gives too few CTAs; costliest first
+    // (head-uniform: one item list for all heads, item.x = tensor)
     std::vector<int4> tci;
-    const int parts_want = std::max(1, (4 * 148 + 2 * d.nblk * c.h - 1) / (2 * d.nblk * c.h));
-    for (int hh = 0; hh < c.h; ++hh)
+    const int hs = c.mode == HTTM_HEAD_UNIFORM ? 1 : c.h;
+    const int parts_want = std::max(1, (4 * 148 + 2 * d.nblk * hs - 1) / (2 * d.nblk * hs));
+    for (int hh = 0; hh < hs; ++hh)
       for (int t = 0; t < 2; ++t)
         for (int bi = 0; bi < d.nblk; ++bi) {
           const BlockDesc& b = B[bi];

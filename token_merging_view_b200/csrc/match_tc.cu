@@ -309,17 +309,261 @@ match_tc_kernel(Dims dims, const BlockDesc* __restrict__ blocks, const int4* __r
   }
 }
 
+
+// Head-uniform variant (one plan per block for every head, ToMe / FastVGGT
+// style; HTTM note, background section): the score of a (source,
+// destination) pair is the mean over heads of the per-head cosines,
+// c(s, t) = (1/h) sum_h dot_h(s, t) / (||s_h|| ||t_h||).  The per-head dot
+// products come from the tensor core on the raw bf16 rows (exact products,
+// fp32 sums) and the per-head norms are applied in the epilogue, so nothing
+// is rounded to bf16 after normalising.  Per (source tile of 128 rows,
+// destination chunk of <= 256 columns) the CTA steps through the heads: the
+// head's source and destination rows are staged in shared memory (double
+// buffered, cp.async), one thread issues S_h = X_s,h X_d,h^T (K = 64) into
+// one of two TMEM buffers, and 16 epilogue warps add S_h * inv_s,h *
+// inv_t,h into register accumulators (a thread: one row, 64 columns); after
+// the last head they take the argmax (strict '>' in ascending column order,
+// lowest index across the four column parts on ties) and keep a running
+// best over the chunks.  The plan is written for every head.
+constexpr int kUChunk = 256;
+
+struct UniformSmem {
+  uint8_t src[2][kRowsTile * 128];            // staged source rows of one head (K-major SW128)
+  uint8_t dst[2][kUChunk * 128];              // staged destination rows of one head
+  float inv_s[2][kRowsTile];
+  float inv_t[2][kUChunk];
+  float best_v[kParts][128];
+  int best_i[kParts][128];
+  uint64_t ready[2], full[2], empty[2], drain;
+  uint32_t tmem_base;
+  int abort;
+};
+constexpr size_t kUSmemBytes = sizeof(UniformSmem) + 1024;
+
+// item: tensor (0 = Q, 1 = K), block, first source ordinal, sources
+__global__ void __launch_bounds__(kThreads, 1)
+match_uniform_tc_kernel(Dims dims, const BlockDesc* __restrict__ blocks, const int4* __restrict__ items,
+                        const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K, Buffers buf) {
+  extern __shared__ uint8_t smem_raw[];
+  UniformSmem& sm = *reinterpret_cast<UniformSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int4 it = items[blockIdx.x];
+  const bool is_q = it.x == 0;
+  const BlockDesc b = blocks[it.y];
+  const int H = dims.h;
+  const int stride = is_q ? dims.q_stride : dims.kv_stride;
+  const int ndst = is_q ? b.q_ndst : b.k_ndst;
+  const int ndst_pad = (ndst + 63) & ~63;
+  const int nchunk = (ndst_pad + kUChunk - 1) / kUChunk;
+  const int src0 = it.z, nsrc = it.w;
+  const int ntile = (nsrc + kRowsTile - 1) / kRowsTile;
+  const int nstep = ntile * nchunk * H;
+  const __nv_bfloat16* X = is_q ? Q : K;
+  const int src_off = is_q ? b.q_src_off : b.k_src_off;
+  const int nsrc_head = is_q ? dims.q_src : dims.k_src;
+  int32_t* best_out = is_q ? buf.q_best : buf.k_best;
+  float* score_out = is_q ? buf.q_score : buf.k_score;
+  DevState* st = buf.state;
+
+  if (tid == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.ready[i], kEpiThreads);
+      mbar_init(&sm.full[i], 1);
+      mbar_init(&sm.empty[i], kEpiThreads);
+    }
+    mbar_init(&sm.drain, 1);
+    sm.abort = 0;
+    mbar_fence_init();
+  }
+  if (warp == kEpiThreads / 32) tmem_alloc(&sm.tmem_base, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* abort = &sm.abort;
+
+  if (warp == kEpiThreads / 32) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ MMA issue
+      for (int s = 0; s < nstep; ++s) {
+        const int bb = s & 1;
+        if (!mbar_wait(&sm.ready[bb], (s >> 1) & 1, abort, st)) break;
+        if (s >= 2 && !mbar_wait(&sm.empty[bb], ((s - 2) >> 1) & 1, abort, st)) break;
+        tc_fence_after();
+        const int c = (s / H) % nchunk;
+        const int width = min(kUChunk, ndst_pad - c * kUChunk);
+        const uint32_t idesc = idesc_bf16(128, width, false, false);
+        const uint32_t sa = smem_u32(sm.src[bb]), da = smem_u32(sm.dst[bb]);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          umma_bf16(tmem + bb * kUChunk, sw128_desc(sa + kk * 32, 1024), sw128_desc(da + kk * 32, 1024), idesc,
+                    kk > 0);
+        umma_commit(&sm.full[bb]);
+      }
+      umma_commit(&sm.drain);
+      drain_wait(&sm.drain, 0);
+    }
+  } else {
+    // ------------------------------------------------------ gather + epilogue
+    // stage step s: head h's source tile and destination chunk
+    auto load_step = [&](int s) {
+      const int bb = s & 1;
+      const int h = s % H, c = (s / H) % nchunk, t = s / (H * nchunk);
+      const __nv_bfloat16* Xh = X + (size_t)h * dims.N * 64;
+      const uint32_t sb = smem_u32(sm.src[bb]), db = smem_u32(sm.dst[bb]);
+      for (int e = tid; e < (int)kRowsTile * 8; e += kEpiThreads) {
+        const int r = e >> 3, ch = e & 7;
+        const int k = src0 + t * kRowsTile + r;
+        const bool valid = t * (int)kRowsTile + r < nsrc;
+        const int tok = valid ? block_token(b, src_index(k, stride), dims.P) : b.base;
+        cp_async16(sb + swz(r, ch), Xh + (size_t)tok * 64 + ch * 8, valid);
+      }
+      for (int e = tid; e < kUChunk * 8; e += kEpiThreads) {
+        const int r = e >> 3, ch = e & 7;
+        const int m = c * kUChunk + r;
+        const bool valid = m < ndst;
+        const int tok = valid ? block_token(b, m * stride, dims.P) : b.base;
+        cp_async16(db + swz(r, ch), Xh + (size_t)tok * 64 + ch * 8, valid);
+      }
+    };
+    auto row_inv = [](const uint8_t* base, int r) {
+      float ss = 0.f;
+      for (int ch = 0; ch < 8; ++ch) {
+        const uint4 w = *reinterpret_cast<const uint4*>(base + swz(r, ch));
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float lo = __uint_as_float(ws[q] << 16), hi = __uint_as_float(ws[q] & 0xffff0000u);
+          ss = fmaf(lo, lo, ss);
+          ss = fmaf(hi, hi, ss);
+        }
+      }
+      return ss > 0.f ? 1.f / sqrtf(ss) : 0.f;
+    };
+    const int quarter = warp & 3, part = warp >> 2;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    bool ok = true;
+    float acc[64];
+    float bv = -INFINITY;
+    int bx = 0x7fffffff;
+    load_step(0);
+    cp_async_commit();
+    for (int s = 0; s < nstep; ++s) {
+      const int bb = s & 1;
+      const int h = s % H, c = (s / H) % nchunk, t = s / (H * nchunk);
+      if (s + 1 < nstep) {
+        load_step(s + 1);           // its buffers were last read by step s - 1, complete below
+        cp_async_commit();
+        cp_async_wait<1>();
+      } else {
+        cp_async_wait<0>();
+      }
+      fence_async_smem();
+      epi_sync();
+      if (tid < kRowsTile) sm.inv_s[bb][tid] = row_inv(sm.src[bb], tid);
+      else if (tid < kRowsTile + kUChunk) sm.inv_t[bb][tid - kRowsTile] = row_inv(sm.dst[bb], tid - kRowsTile);
+      epi_sync();
+      mbar_arrive(&sm.ready[bb]);
+      if (h == 0) {
+#pragma unroll
+        for (int e = 0; e < 64; ++e) acc[e] = 0.f;
+      }
+      const int width = min(kUChunk, ndst_pad - c * kUChunk);
+      if (ok && !__all_sync(0xffffffffu, mbar_wait(&sm.full[bb], (s >> 1) & 1, abort, st))) {
+        ok = false;
+        *abort = 1;
+      }
+      if (ok) {
+        tc_fence_after();
+        const int g0 = part * 64;
+        if (g0 < width) {
+          const float is = sm.inv_s[bb][row];
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            uint32_t r0[32];
+            tmem_ld32(tmem + lane_off + bb * kUChunk + g0 + half * 32, r0);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              acc[half * 32 + e] = fmaf(__uint_as_float(r0[e]) * is, sm.inv_t[bb][g0 + half * 32 + e], acc[half * 32 + e]);
+          }
+        }
+        tc_fence_before();
+      }
+      mbar_arrive(&sm.empty[bb]);
+      if (h == H - 1) {
+        // the chunk's mean cosines: this part's argmax joins the running best
+        const float inv_h = 1.f / (float)H;
+        const int cb = c * kUChunk + part * 64;
+#pragma unroll
+        for (int e = 0; e < 64; ++e) {
+          const float v = acc[e] * inv_h;
+          if (cb + e < ndst && v > bv) {
+            bv = v;
+            bx = cb + e;
+          }
+        }
+        if (c == nchunk - 1) {
+          // the tile is done: combine the four column parts of each row
+          sm.best_v[part][row] = bv;
+          sm.best_i[part][row] = bx;
+          epi_sync();
+          if (part == 0 && ok) {
+            const int k = t * kRowsTile + row;
+            if (k < nsrc) {
+              float v = sm.best_v[0][row];
+              int i = sm.best_i[0][row];
+#pragma unroll
+              for (int p = 1; p < kParts; ++p) {
+                const float v1 = sm.best_v[p][row];
+                const int i1 = sm.best_i[p][row];
+                if (v1 > v || (v1 == v && i1 < i)) {
+                  v = v1;
+                  i = i1;
+                }
+              }
+              for (int hh = 0; hh < H; ++hh) {
+                best_out[(size_t)hh * nsrc_head + src_off + src0 + k] = i;
+                score_out[(size_t)hh * nsrc_head + src_off + src0 + k] = v;
+              }
+            }
+          }
+          epi_sync();
+          bv = -INFINITY;
+          bx = 0x7fffffff;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kEpiThreads / 32) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 }  // namespace
 
 bool tma_encode_available();
 
 bool match_tc_supported(const Dims& dims, bool fp32) {
-  return !fp32 && dims.d == 64 && dims.mode != HTTM_HEAD_UNIFORM && dims.max_ndst <= kMaxDst;
+  return !fp32 && dims.d == 64 && dims.max_ndst <= kMaxDst;
 }
 
 cudaError_t launch_match_tc(const Dims& dims, const BlockDesc* blocks, const int4* items, int n_items,
                             const void* Q, const void* K, const Buffers& buf, cudaStream_t s) {
   if (n_items == 0) return cudaSuccess;
+  if (dims.mode == HTTM_HEAD_UNIFORM) {
+    cudaError_t e = cudaFuncSetAttribute(match_uniform_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kUSmemBytes);
+    if (e != cudaSuccess) return e;
+    match_uniform_tc_kernel<<<n_items, kThreads, kUSmemBytes, s>>>(
+        dims, blocks, items, static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K), buf);
+    return cudaGetLastError();
+  }
   cudaError_t e = cudaFuncSetAttribute(match_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   match_tc_kernel<<<n_items, kThreads, kSmemBytes, s>>>(
