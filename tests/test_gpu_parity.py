@@ -233,3 +233,11 @@ def test_short_key_ranges_split_parts(T):
         assert torch.equal(o, outs[0])
     mx, rl2 = PL.sample_out_error(res, PL.to64(outs[0]), cfg, 1 << 30)
     assert mx <= PL.OUT_MAX_ABS and rl2 <= PL.OUT_REL_L2, (mx, rl2)
+
+
+@pytest.mark.slow
+def test_vggt_30f_head_uniform_plan():
+    """The head-uniform plan at the 30-frame layer's shape (16 heads, blocks
+    of 3840 / 2670 tokens) from the tensor-core matcher: the plan against the
+    oracle's, and the output on the oracle's plan and mask."""
+    _full_check(WORKLOADS["vggt_30f"].with_(mode=HEAD_UNIFORM), tokens_per_head=256)
