@@ -29,7 +29,7 @@ The mean update is the same as LiteVGGT's x_d <- (x_d + sum_{s in S_d} x_s) /
 (1 + |S_d|) ("LiteVGGT: Boosting Vanilla VGGT via Geometry-aware Cached Token
 Merging", key design 3).
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent:
 
 * spatial regions are contiguous raster ranges of the patch index p, the last
   one partial; temporal groups are runs of n_t frames, the last one partial;
