@@ -241,3 +241,10 @@ def test_vggt_30f_head_uniform_plan():
     of 3840 / 2670 tokens) from the tensor-core matcher: the plan against the
     oracle's, and the output on the oracle's plan and mask."""
     _full_check(WORKLOADS["vggt_30f"].with_(mode=HEAD_UNIFORM), tokens_per_head=256)
+
+
+@pytest.mark.parametrize("kw", [dict(d=16), dict(fp32=True, T=3, h=2)], ids=["bf16_d16", "fp32_d64"])
+def test_mid_layer_cuda_core_paths(kw):
+    """Shapes served by the CUDA-core matching and attention kernels (bf16
+    with d_head = 16, fp32 with d_head = 64) against the oracle."""
+    _full_check(MID.with_(**kw))
