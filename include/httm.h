@@ -225,6 +225,19 @@ httm_status httm_forward_reuse(httm_plan_t plan, const void* Q, const void* K, c
 httm_status httm_reorder(httm_plan_t plan, const void* X, void* Xb, int inverse, void* stream);
 
 /*
+ * httm_set_wait_budget: the bound, in nanoseconds, of every device-side wait
+ * of the later forward calls on `plan` (default 2e9: 2 s).  A wait that runs
+ * out sets HTTM_DEV_TIMEOUT in the status word; its CTA stops its work,
+ * waits (with a fixed 2 s bound) for the tensor-core operations it issued,
+ * frees its tensor memory and exits, and the call's output is undefined.
+ * The context stays usable.  0 makes every wait that is not already
+ * complete run out at once: a failure-detection check, not a setting for
+ * real work.  Host only; returns HTTM_ERR_ARG for a null plan.  Not from the
+ * pages (bounded waits are this library's own safeguard).
+ */
+httm_status httm_set_wait_budget(httm_plan_t plan, uint64_t nanoseconds);
+
+/*
  * Synchronises `stream`, then reads the device status word of `workspace`
  * into *status (0 = clean; HTTM_DEV_* bits otherwise) and clears it.
  * Returns HTTM_ERR_DEVICE_BOUNDS / HTTM_ERR_TIMEOUT when bits were set.

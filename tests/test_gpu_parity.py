@@ -248,3 +248,21 @@ def test_mid_layer_cuda_core_paths(kw):
     """Shapes served by the CUDA-core matching and attention kernels (bf16
     with d_head = 16, fp32 with d_head = 64) against the oracle."""
     _full_check(MID.with_(**kw))
+
+
+@pytest.mark.parametrize("w", [MID, MID.with_(mode=HEAD_UNIFORM)], ids=["headwise", "head_uniform"])
+def test_wait_that_runs_out_sets_timeout_and_context_recovers(w):
+    """Failure detection without a fault: with a zero wait budget the first
+    device wait that is not already complete gives up, the status word says
+    HTTM_DEV_TIMEOUT, the kernels free what they hold and exit; with the
+    default budget restored the same plan gives the same bits as before."""
+    _, plan, _, (Q, K, V), _ = _case(w)
+    ref = B.httm_forward(plan, Q, K, V, workspace=plan.new_workspace())
+    ws = plan.new_workspace()
+    B.httm_set_wait_budget(plan, 0)
+    B.httm_forward(plan, Q, K, V, workspace=ws)
+    assert B.httm_get_device_status(plan, ws) & B.HTTM_DEV_TIMEOUT
+    B.httm_set_wait_budget(plan, 2_000_000_000)
+    again = B.httm_forward(plan, Q, K, V, workspace=ws)
+    assert B.httm_get_device_status(plan, ws) == 0
+    assert torch.equal(again, ref)

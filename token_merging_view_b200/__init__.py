@@ -19,6 +19,7 @@ from .binding import (  # noqa: F401
     httm_get_device_status,
     httm_plan,
     httm_reorder,
+    httm_set_wait_budget,
     load_library,
     workspace_view,
 )

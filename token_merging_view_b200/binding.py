@@ -26,7 +26,7 @@ EXPORTS = (
     "httm_plan", "httm_plan_destroy", "httm_get_plan_info", "httm_workspace_bytes",
     "httm_forward", "httm_forward_debug", "httm_forward_with_plan", "httm_forward_reuse", "httm_reorder",
     "httm_get_device_status", "httm_forward_launches", "httm_profile_enable", "httm_profile_read",
-    "httm_select_outliers_noalloc", "httm_status_str",
+    "httm_select_outliers_noalloc", "httm_set_wait_budget", "httm_status_str",
 )
 STAGES = ("match", "merge", "outlier", "attention", "unmerge", "other")
 
@@ -91,6 +91,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.httm_profile_read.argtypes = [P, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int32)]
     lib.httm_select_outliers_noalloc.argtypes = [V, V, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, V, V, V]
     lib.httm_select_outliers_noalloc.restype = ctypes.c_int
+    lib.httm_set_wait_budget.argtypes = [P, ctypes.c_uint64]
+    lib.httm_set_wait_budget.restype = ctypes.c_int
     lib.httm_status_str.argtypes = [I]
     lib.httm_status_str.restype = ctypes.c_char_p
     for name in ("httm_plan", "httm_get_plan_info", "httm_forward", "httm_forward_debug",
@@ -286,6 +288,13 @@ def httm_reorder(plan: Plan, X, inverse: bool = False, out=None, stream=None):
     _check(load_library().httm_reorder(plan.handle, _ptr(X), _ptr(out), int(inverse), _stream(stream)),
            "httm_reorder")
     return out
+
+
+def httm_set_wait_budget(plan: Plan, nanoseconds: int) -> None:
+    """Bound of every device-side wait of later forward calls on ``plan``
+    (default 2e9 ns); 0 makes every wait that is not already complete run
+    out (HTTM_DEV_TIMEOUT), for checking the failure path."""
+    _check(load_library().httm_set_wait_budget(plan.handle, int(nanoseconds)), "httm_set_wait_budget")
 
 
 def httm_get_device_status(plan: Plan, workspace, stream=None) -> int:

@@ -358,6 +358,7 @@ httm_status httm_plan(const httm_cfg* cfg, httm_plan_t* out) {
   d.scale = c.softmax_scale > 0.f ? c.softmax_scale : 1.0f / sqrtf((float)c.d_head);
   d.plan_id = next_id.fetch_add(1);
   if (d.plan_id == 0) d.plan_id = next_id.fetch_add(1);
+  d.wait_budget_ns = 2000000000ull;
   d.nchunk_per_head = (int32_t)((N + kChunk - 1) / kChunk);
   if (c.mode == HTTM_DENSE) {
     d.max_items = (int32_t)(c.h * ((N + kAttnRows - 1) / kAttnRows));
@@ -555,6 +556,12 @@ httm_status httm_get_device_status(httm_plan_t plan, void* workspace, void* stre
 }
 
 int32_t httm_forward_launches(httm_plan_t plan) { return plan ? plan->launches : -1; }
+
+httm_status httm_set_wait_budget(httm_plan_t plan, uint64_t nanoseconds) {
+  if (!plan) return HTTM_ERR_ARG;
+  plan->dims.wait_budget_ns = nanoseconds;
+  return HTTM_OK;
+}
 
 httm_status httm_profile_enable(httm_plan_t plan, int enable) {
   if (!plan) return HTTM_ERR_ARG;

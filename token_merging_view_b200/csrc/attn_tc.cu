@@ -76,7 +76,7 @@ static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 
 // Bounded wait that ignores the abort flag (used to drain in-flight MMAs).
 __device__ bool drain_wait(uint64_t* bar, uint32_t parity) {
-  const WaitClock clk;
+  const WaitClock clk;                                // the fixed 2 s bound, whatever the call's budget
   while (!mbar_try_wait(bar, parity))
     if (clk.expired()) return false;
   return true;

@@ -38,6 +38,7 @@ struct Dims {
   int32_t max_items;             // attention work items (upper bound)
   float scale;
   uint32_t plan_id;              // stamps a workspace whose member lists this plan wrote
+  uint64_t wait_budget_ns;       // bound of a device wait (httm_set_wait_budget; default 2 s)
 };
 
 constexpr int kChunk = 4096;       // keys per chunk of the outlier compaction
@@ -58,6 +59,7 @@ struct DevState {
   uint32_t wait_cta;             // ... its CTA index
   uint32_t wait_grid;            // ... and the grid size of its launch (tells the kernels apart)
   uint32_t pad_;
+  uint64_t wait_ns;              // this call's wait bound (from Dims::wait_budget_ns)
 };
 
 struct Workspace {

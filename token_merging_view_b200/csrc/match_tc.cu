@@ -67,7 +67,7 @@ __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_gr
 __device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory"); }
 
 __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
-  const WaitClock clk;
+  const WaitClock clk;                                // the fixed 2 s bound, whatever the call's budget
   while (!mbar_try_wait(bar, parity))
     if (clk.expired()) return false;
   return true;

@@ -792,7 +792,7 @@ __global__ void export_kernel(Dims dims, const BlockDesc* __restrict__ blocks, B
   }
 }
 
-__global__ void zero_state_kernel(Buffers buf, int keep_stamp) {
+__global__ void zero_state_kernel(Buffers buf, int keep_stamp, unsigned long long wait_ns) {
   for (int i = threadIdx.x; i < 3 * kHistBins; i += blockDim.x) buf.hist[i] = 0u;
   if (threadIdx.x == 0) {
     if (!keep_stamp) buf.state->plan_stamp = 0u;   // rewritten once this call's planning has succeeded
@@ -802,6 +802,7 @@ __global__ void zero_state_kernel(Buffers buf, int keep_stamp) {
     buf.state->wait_site = 0u;
     buf.state->wait_cta = 0u;
     buf.state->wait_grid = 0u;
+    buf.state->wait_ns = wait_ns;
   }
   if (threadIdx.x < 8) buf.state->sel[threadIdx.x] = 0u;
 }
@@ -836,8 +837,8 @@ cudaError_t launch_merge_t(const Dims& dims, const BlockDesc* blocks, bool injec
 
 }  // namespace
 
-cudaError_t launch_zero_state(const Dims&, const Buffers& buf, bool keep_stamp, cudaStream_t s) {
-  zero_state_kernel<<<1, 1024, 0, s>>>(buf, keep_stamp ? 1 : 0);
+cudaError_t launch_zero_state(const Dims& dims, const Buffers& buf, bool keep_stamp, cudaStream_t s) {
+  zero_state_kernel<<<1, 1024, 0, s>>>(buf, keep_stamp ? 1 : 0, (unsigned long long)dims.wait_budget_ns);
   return cudaGetLastError();
 }
 

@@ -24,7 +24,6 @@ namespace httm {
 namespace tc {
 
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s for any single wait inside a CTA
-constexpr unsigned long long kWaitTimeoutCycles = 2000000000ull;  // ~1 s at the 1965 MHz top SM clock
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -46,14 +45,15 @@ __device__ __forceinline__ unsigned long long sm_cycles() {
 // SM's cycle counter.  The global timer is kept in step with the host clock
 // by the driver and may move forward in a jump; the cycle counter cannot
 // jump but runs slower at low clocks.  A wait ends only when both say it has
-// gone on too long (>= kWaitTimeoutNs of global time and >= 1 s worth of
-// cycles at the top SM clock), so it stays bounded (a few seconds at most)
-// and a timer jump alone does not end it.
+// gone on too long (more than `budget` ns of global time and more than
+// `budget` cycles: with the default 2e9, 2 s and ~1 s at the 1965 MHz top SM
+// clock), so it stays bounded and a timer jump alone does not end it.
 struct WaitClock {
-  unsigned long long ns0, cyc0;
-  __device__ __forceinline__ WaitClock() : ns0(globaltimer()), cyc0(sm_cycles()) {}
+  unsigned long long ns0, cyc0, budget;
+  __device__ __forceinline__ explicit WaitClock(unsigned long long budget_ns = kWaitTimeoutNs)
+      : ns0(globaltimer()), cyc0(sm_cycles()), budget(budget_ns) {}
   __device__ __forceinline__ bool expired() const {
-    return globaltimer() - ns0 > kWaitTimeoutNs && sm_cycles() - cyc0 > kWaitTimeoutCycles;
+    return globaltimer() - ns0 > budget && sm_cycles() - cyc0 > budget;
   }
 };
 
@@ -108,11 +108,11 @@ __device__ __forceinline__ void record_timeout(DevState* st, uint64_t* bar, uint
 }
 
 // Waits for the phase of `parity` to complete.  Gives up when its WaitClock
-// expires or when *abort is set: then it sets *abort and the
+// (the call's budget, DevState::wait_ns) expires or when *abort is set: then it sets *abort and the
 // HTTM_DEV_TIMEOUT status bit and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, DevState* st) {
   if (mbar_try_wait(bar, parity)) return true;
-  const WaitClock clk;
+  const WaitClock clk(st->wait_ns);
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
