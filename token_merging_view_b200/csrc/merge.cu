@@ -517,20 +517,55 @@ gather_kernel(Dims dims, const T* __restrict__ X, const T* __restrict__ V, Buffe
       }
       if (IS_Q) {
         for (int q0 = 0; q0 < cmax; q0 += kU) {
+          if constexpr (CPR == 8 && kU == 4) {
+            // four members at once: each lane's partial sums of squares,
+            // then a reduce-scatter over the row's 8 lanes (xor 4, 2, 1)
+            // that leaves member m's sum in lanes 2m' (m = 2 bit2 + bit1 of
+            // the lane), whose even lanes then write the four keys together
+            int tok[kU];
+            float s4[kU];
 #pragma unroll
-          for (int u = 0; u < kU; ++u) {
-            const int q = q0 + u;
-            const bool mine = q < c_cur;
-            const int tok = q0 == 0 ? tk0[u] : (mine ? members[tokbase + gs_cur + q] : 0);
-            uint4 xr = xk[u];
-            if (q0 > 0 && mine) xr = Ch::load(Xh + (size_t)tok * D, ch);
-            const float ss = Ch::within_row(mine && c_cur >= 2 ? Ch::sq_dist(xr, acc) : 0.f);
-            if (mine && ch == 0) {
+            for (int u = 0; u < kU; ++u) {
+              const int q = q0 + u;
+              const bool mine = q < c_cur;
+              tok[u] = q0 == 0 ? tk0[u] : (mine ? members[tokbase + gs_cur + q] : 0);
+              uint4 xr = xk[u];
+              if (q0 > 0 && mine) xr = Ch::load(Xh + (size_t)tok[u] * D, ch);
+              s4[u] = mine && c_cur >= 2 ? Ch::sq_dist(xr, acc) : 0.f;
+            }
+            const bool b2 = (ch & 4) != 0, b1 = (ch & 2) != 0;
+            float k0 = b2 ? s4[2] : s4[0], k1 = b2 ? s4[3] : s4[1];
+            k0 += __shfl_xor_sync(0xffffffffu, b2 ? s4[0] : s4[2], 4);
+            k1 += __shfl_xor_sync(0xffffffffu, b2 ? s4[1] : s4[3], 4);
+            float ss = b1 ? k1 : k0;
+            ss += __shfl_xor_sync(0xffffffffu, b1 ? k0 : k1, 2);
+            ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+            const int m = (b2 ? 2 : 0) + (b1 ? 1 : 0);
+            if ((ch & 1) == 0 && q0 + m < c_cur) {
+              const int tm = m == 0 ? tok[0] : m == 1 ? tok[1] : m == 2 ? tok[2] : tok[3];
               const uint32_t key = c_cur >= 2 ? __float_as_uint(sqrtf(ss)) + 1u : 0u;
-              buf.keys[tokbase + tok] = key;
+              buf.keys[tokbase + tm] = key;
               if (key) {
                 atomicAdd(&hist[key >> 21], 1u);
                 ++elig;
+              }
+            }
+          } else {
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+              const int q = q0 + u;
+              const bool mine = q < c_cur;
+              const int tok = q0 == 0 ? tk0[u] : (mine ? members[tokbase + gs_cur + q] : 0);
+              uint4 xr = xk[u];
+              if (q0 > 0 && mine) xr = Ch::load(Xh + (size_t)tok * D, ch);
+              const float ss = Ch::within_row(mine && c_cur >= 2 ? Ch::sq_dist(xr, acc) : 0.f);
+              if (mine && ch == 0) {
+                const uint32_t key = c_cur >= 2 ? __float_as_uint(sqrtf(ss)) + 1u : 0u;
+                buf.keys[tokbase + tok] = key;
+                if (key) {
+                  atomicAdd(&hist[key >> 21], 1u);
+                  ++elig;
+                }
               }
             }
           }
