@@ -25,6 +25,11 @@ struct httm_plan_s {
   int n_match_items = 0;
   int4* tc_items_d = nullptr;   // tensor-core matching: (tensor + 2 * head, block, first source, sources)
   int n_tc_items = 0;
+  int n_tc_q = 0;               // the query items come first in tc_items
+  // the key branch of a forward (matching, planning and gathering K/V) runs
+  // on this stream, beside the query branch on the caller's stream
+  cudaStream_t side = nullptr;
+  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
   std::vector<int4> tc_items_h;
   Workspace ws;
   int launches = 0;
@@ -191,6 +196,17 @@ httm_status check_device(httm_plan_s* plan) {
         return HTTM_ERR_CUDA;
       }
     }
+    if (plan->dims.mode != HTTM_DENSE &&
+        (cudaStreamCreateWithFlags(&plan->side, cudaStreamNonBlocking) != cudaSuccess ||
+         cudaEventCreateWithFlags(&plan->ev_fork, cudaEventDisableTiming) != cudaSuccess ||
+         cudaEventCreateWithFlags(&plan->ev_join, cudaEventDisableTiming) != cudaSuccess)) {
+      if (plan->side) cudaStreamDestroy(plan->side);
+      if (plan->ev_fork) cudaEventDestroy(plan->ev_fork);
+      if (plan->ev_join) cudaEventDestroy(plan->ev_join);
+      plan->side = nullptr;
+      plan->ev_fork = plan->ev_join = nullptr;
+      return HTTM_ERR_CUDA;
+    }
     plan->device = dev;
   }
   return dev == plan->device ? HTTM_OK : HTTM_ERR_ARG;
@@ -263,6 +279,38 @@ httm_status forward_impl(httm_plan_s* plan, const void* Q, const void* K, const 
     StageTimer t(plan, s, HTTM_STAGE_OTHER, 1);
     Inject ii{inj->q_best, inj->q_merged, inj->k_best, inj->k_merged, inj->outlier};
     HTTM_LAUNCH(launch_import_plan(dims, plan->blocks_d, ii, buf, s));
+  }
+  // Without stage timing, the key branch (matching, planning and the K/V
+  // gather) runs on the plan's side stream beside the query branch
+  // (matching, planning, the query gather and the outlier filter), joined
+  // before attention: the branches share no buffer, and the small,
+  // latency-bound kernels of one overlap the other's.  With stage timing
+  // everything runs in order on `s`, so that each stage can be timed.
+  if (!plan->profile && plan->side && match_tc_supported(dims, fp32)) {
+    cudaStream_t s2 = plan->side;
+    if (cudaEventRecord(plan->ev_fork, s) != cudaSuccess || cudaStreamWaitEvent(s2, plan->ev_fork, 0) != cudaSuccess)
+      return HTTM_ERR_CUDA;
+    if (!plan_inj && !reuse) {
+      if (plan->n_tc_q > 0)
+        HTTM_LAUNCH(launch_match_tc(dims, plan->blocks_d, plan->tc_items_d, plan->n_tc_q, Q, K, buf, s));
+      if (plan->n_tc_items > plan->n_tc_q)
+        HTTM_LAUNCH(launch_match_tc(dims, plan->blocks_d, plan->tc_items_d + plan->n_tc_q,
+                                    plan->n_tc_items - plan->n_tc_q, Q, K, buf, s2));
+    }
+    HTTM_LAUNCH(launch_merge(dims, fp32, plan->blocks_d, plan_inj, reuse, Q, K, V, buf, dd, s, 1));
+    HTTM_LAUNCH(launch_merge(dims, fp32, plan->blocks_d, plan_inj, reuse, Q, K, V, buf, dd, s2, 2));
+    if (!reuse) launches += 2;  // the two planning launches
+    HTTM_LAUNCH(launch_outlier(dims, fp32, Q, mask_inj, buf, s));
+    launches += mask_inj ? 2 : 4;
+    HTTM_LAUNCH(launch_restore(dims, fp32, plan->blocks_d, Q, buf, dd, s));
+    if (cudaEventRecord(plan->ev_join, s2) != cudaSuccess || cudaStreamWaitEvent(s, plan->ev_join, 0) != cudaSuccess)
+      return HTTM_ERR_CUDA;
+    st = attention(plan, buf.q_tilde, buf.k_tilde, buf.v_tilde, buf.o_tilde, dims.k_slots, buf, s, &launches);
+    if (st != HTTM_OK) return st;
+    HTTM_LAUNCH(launch_unmerge(dims, fp32, buf, out, s));
+    if (dbg) HTTM_LAUNCH(launch_export(dims, plan->blocks_d, buf, dd, s));
+    plan->launches = launches;
+    return HTTM_OK;
   }
   if (!plan_inj && !reuse) {
     StageTimer t(plan, s, HTTM_STAGE_MATCH, 1);
@@ -460,11 +508,14 @@ httm_status httm_plan(const httm_cfg* cfg, httm_plan_t* out) {
             tci.push_back(make_int4(t + 2 * hh, bi, s0, n));
           }
         }
+    // query items first, then key items; each costliest first
     std::stable_sort(tci.begin(), tci.end(), [&](const int4& a, const int4& b) {
+      if ((a.x & 1) != (b.x & 1)) return (a.x & 1) < (b.x & 1);
       const long long ca = (long long)((a.x & 1) == 0 ? B[a.y].q_ndst : B[a.y].k_ndst) * a.w;
       const long long cb = (long long)((b.x & 1) == 0 ? B[b.y].q_ndst : B[b.y].k_ndst) * b.w;
       return ca > cb;
     });
+    p->n_tc_q = (int)std::count_if(tci.begin(), tci.end(), [](const int4& a) { return (a.x & 1) == 0; });
     p->n_tc_items = (int)tci.size();
     p->tc_items_h = std::move(tci);
   }
@@ -483,6 +534,9 @@ void httm_plan_destroy(httm_plan_t plan) {
   if (plan->blocks_d) cudaFree(plan->blocks_d);
   if (plan->match_items_d) cudaFree(plan->match_items_d);
   if (plan->tc_items_d) cudaFree(plan->tc_items_d);
+  if (plan->side) cudaStreamDestroy(plan->side);
+  if (plan->ev_fork) cudaEventDestroy(plan->ev_fork);
+  if (plan->ev_join) cudaEventDestroy(plan->ev_join);
   delete plan;
 }
 

@@ -38,12 +38,13 @@ cudaError_t launch_match_tc(const Dims& dims, const BlockDesc* blocks, const int
 cudaError_t launch_import_plan(const Dims& dims, const BlockDesc* blocks, const Inject& inj,
                                const Buffers& buf, cudaStream_t s);
 
-// Merge planning (Q and K) then the mean-merging gathers of Q and of K/V:
-// three launches; with `reuse`, only the gathers, on the member lists an
-// earlier call left in the workspace.
+// Merge planning then the mean-merging gathers; `tensors` 3: Q and K (the
+// planning of both in one launch, then the Q gather and the K/V gather),
+// 1: Q only, 2: K (and V) only.  With `reuse`, only the gathers, on the
+// member lists an earlier call left in the workspace.
 cudaError_t launch_merge(const Dims& dims, bool fp32, const BlockDesc* blocks, bool injected, bool reuse,
                          const void* Q, const void* K, const void* V, const Buffers& buf,
-                         const Debug& dbg, cudaStream_t s);
+                         const Debug& dbg, cudaStream_t s, int tensors = 3);
 
 cudaError_t launch_outlier(const Dims& dims, bool fp32, const void* Q, bool mask_injected,
                            const Buffers& buf, cudaStream_t s);

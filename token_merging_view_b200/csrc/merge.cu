@@ -213,7 +213,8 @@ struct SmallDiv {
 // the member list written position by position (a binary search over the
 // group starts finds each position's group).
 __global__ void __launch_bounds__(kMergeThreads)
-plan_kernel(Dims dims, const BlockDesc* __restrict__ blocks, Buffers buf, Debug dbg, int injected, int cap) {
+plan_kernel(Dims dims, const BlockDesc* __restrict__ blocks, Buffers buf, Debug dbg, int injected, int cap,
+            int tensor0) {
   extern __shared__ __align__(16) unsigned char smem[];
   uint32_t* key = reinterpret_cast<uint32_t*>(smem);        // [cap] ordered score bits
   int32_t* bst = reinterpret_cast<int32_t*>(key + cap);      // [cap] destination of each source
@@ -229,7 +230,7 @@ plan_kernel(Dims dims, const BlockDesc* __restrict__ blocks, Buffers buf, Debug 
   __shared__ int s_bin;
   __shared__ uint32_t s_krem;
 
-  const bool is_q = blockIdx.z == 0;
+  const bool is_q = blockIdx.z + tensor0 == 0;         // z-th tensor from tensor0 (0 = Q, 1 = K)
   const int tid = threadIdx.x, bd = blockDim.x;
   const int hh = blockIdx.y;
   const BlockDesc b = blocks[blockIdx.x];
@@ -851,22 +852,26 @@ int gather_grid(long long units, int per_sm = 8) {
 
 template <class T, int D>
 cudaError_t launch_merge_t(const Dims& dims, const BlockDesc* blocks, bool injected, bool reuse, const void* Q,
-                           const void* K, const void* V, const Buffers& buf, const Debug& dbg, cudaStream_t s) {
+                           const void* K, const void* V, const Buffers& buf, const Debug& dbg, cudaStream_t s,
+                           int tensors) {
+  const bool do_q = (tensors & 1) != 0, do_k = (tensors & 2) != 0;
   if (!reuse) {
     // cap sources per block, and 2 * cap >= n_b for the position map
     const int cap = (std::max(dims.max_nsrc, (dims.max_nb + 1) / 2) + kMergeThreads - 1) / kMergeThreads * kMergeThreads;
     const size_t smem = (size_t)cap * 17 + 3ull * dims.max_ndst * 4 + 256 * 4 + 64 * 4;
     cudaError_t e = cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    plan_kernel<<<dim3(dims.nblk, dims.h, 2), kMergeThreads, smem, s>>>(dims, blocks, buf, dbg, injected ? 1 : 0,
-                                                                        cap);
+    plan_kernel<<<dim3(dims.nblk, dims.h, (do_q && do_k) ? 2 : 1), kMergeThreads, smem, s>>>(
+        dims, blocks, buf, dbg, injected ? 1 : 0, cap, do_q ? 0 : 1);
   }
   constexpr int RPI = Chunk<T, D>::RPI;
   // resident warps handle several slots each, so that prefetching pays
-  gather_kernel<T, D, true><<<gather_grid((long long)dims.h * dims.q_slots / (4 * RPI) + 1, 4), 256, 0, s>>>(
-      dims, (const T*)Q, nullptr, buf, dbg, reuse ? 1 : 0);
-  gather_kernel<T, D, false><<<gather_grid((long long)dims.h * dims.k_slots / (4 * RPI) + 1, 4), 256, 0, s>>>(
-      dims, (const T*)K, (const T*)V, buf, dbg, reuse ? 1 : 0);
+  if (do_q)
+    gather_kernel<T, D, true><<<gather_grid((long long)dims.h * dims.q_slots / (4 * RPI) + 1, 4), 256, 0, s>>>(
+        dims, (const T*)Q, nullptr, buf, dbg, reuse ? 1 : 0);
+  if (do_k)
+    gather_kernel<T, D, false><<<gather_grid((long long)dims.h * dims.k_slots / (4 * RPI) + 1, 4), 256, 0, s>>>(
+        dims, (const T*)K, (const T*)V, buf, dbg, reuse ? 1 : 0);
   return cudaGetLastError();
 }
 
@@ -879,13 +884,14 @@ cudaError_t launch_zero_state(const Dims& dims, const Buffers& buf, bool keep_st
 
 cudaError_t launch_merge(const Dims& dims, bool fp32, const BlockDesc* blocks, bool injected, bool reuse,
                          const void* Q, const void* K, const void* V, const Buffers& buf, const Debug& dbg,
-                         cudaStream_t s) {
+                         cudaStream_t s, int tensors) {
   if (fp32) {
-    if (dims.d == 16) return launch_merge_t<float, 16>(dims, blocks, injected, reuse, Q, K, V, buf, dbg, s);
-    return launch_merge_t<float, 64>(dims, blocks, injected, reuse, Q, K, V, buf, dbg, s);
+    if (dims.d == 16) return launch_merge_t<float, 16>(dims, blocks, injected, reuse, Q, K, V, buf, dbg, s, tensors);
+    return launch_merge_t<float, 64>(dims, blocks, injected, reuse, Q, K, V, buf, dbg, s, tensors);
   }
-  if (dims.d == 16) return launch_merge_t<__nv_bfloat16, 16>(dims, blocks, injected, reuse, Q, K, V, buf, dbg, s);
-  return launch_merge_t<__nv_bfloat16, 64>(dims, blocks, injected, reuse, Q, K, V, buf, dbg, s);
+  if (dims.d == 16)
+    return launch_merge_t<__nv_bfloat16, 16>(dims, blocks, injected, reuse, Q, K, V, buf, dbg, s, tensors);
+  return launch_merge_t<__nv_bfloat16, 64>(dims, blocks, injected, reuse, Q, K, V, buf, dbg, s, tensors);
 }
 
 cudaError_t launch_restore(const Dims& dims, bool fp32, const BlockDesc*, const void* Q, const Buffers& buf,
