@@ -119,8 +119,9 @@ typedef struct {
  * some block.  The first httm_forward* / httm_reorder call uploads the
  * table to the then-current device (a synchronous copy; make that first call
  * outside any stream capture) and binds the plan to that device: calls from
- * another device return HTTM_ERR_ARG.  The plan owns the table until
- * httm_plan_destroy().
+ * another device return HTTM_ERR_ARG.  That call also creates, except for
+ * HTTM_DENSE, one non-blocking CUDA stream and two events, which the plan
+ * owns with the table until httm_plan_destroy().
  */
 httm_status httm_plan(const httm_cfg* cfg, httm_plan_t* out);
 void httm_plan_destroy(httm_plan_t plan);
@@ -139,7 +140,12 @@ size_t httm_workspace_bytes(httm_plan_t plan);
  * reorder.  Q, K, V: [h, N, d] inputs; out: [h, N, d] output (same dtype).
  * HTTM_DENSE computes plain attention of Q, K, V.  Asynchronous on `stream`;
  * the workspace must not be shared by calls that overlap on the GPU.
- * Bit-deterministic for identical inputs.
+ * Bit-deterministic for identical inputs.  Unless stage timing is on, the
+ * key branch (matching, planning and gathering K/V) runs on the plan's own
+ * stream, forked from `stream` by an event at the call's start and joined
+ * back before attention, so the call stays ordered on `stream` and records
+ * into a CUDA graph captured on it; calls on one plan from several streams
+ * at once share that stream, which only serialises their key branches.
  */
 httm_status httm_forward(httm_plan_t plan, const void* Q, const void* K, const void* V,
                          void* out, void* workspace, size_t workspace_bytes, void* stream);
@@ -255,6 +261,7 @@ int32_t httm_forward_launches(httm_plan_t plan);
  * their elapsed times per stage into ms[HTTM_NUM_STAGES] (milliseconds) and
  * the number of timed launches into launches[HTTM_NUM_STAGES], then forgets
  * them.  Either output may be NULL.  Host-side only; the plan owns the events.
+ * While enabled, every stage runs on `stream` alone, one after another.
  */
 typedef enum {
   HTTM_STAGE_MATCH = 0,     /* bipartite cosine matching (key design 1) */
