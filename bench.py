@@ -33,7 +33,7 @@ METRIC = "merged global-attn layer tokens/s at 100/500 frames; % of HBM & tensor
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="vggt_100f")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -136,6 +136,8 @@ class Clocks:
                                          stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
+        if self.proc is not None:
+            time.sleep(0.3)   # let the sampler start before the timed region does
 
     def stop(self):
         if self.proc is None:
@@ -246,13 +248,14 @@ def measure_layer(w, steps: int, warmup: int, rank: int, world: int, dev, with_e
     clocks = Clocks(dev.index if dev.index is not None else 0)
     total_ms = timed(step, steps)
     clk = clocks.stop()
+    launches = plan.launches() * steps
     plan.profile(True)
     plan.profile_read()
     timed(step, steps)
     stages = plan.profile_read()
     plan.profile(False)
     res = {"plan": plan, "Q": Q, "K": K, "V": V, "ms_step": total_ms / steps, "stages": stages, "sum_lq": sum_lq,
-           "launches": plan.launches() * steps, "clocks": clk}
+           "launches": launches, "clocks": clk}
     if with_e2e:
         # Cached merge indices (LiteVGGT note, key design 3): the following
         # layers reuse the member lists the last full call left in `ws`.
@@ -264,12 +267,13 @@ def measure_layer(w, steps: int, warmup: int, rank: int, world: int, dev, with_e
         torch.cuda.synchronize()
         assert B.httm_get_device_status(plan, ws) == 0
         reuse_ms = timed(reuse, steps) / steps
+        reuse_launches = plan.launches()
         plan.profile(True)
         plan.profile_read()
         timed(reuse, steps)
         rstages = plan.profile_read()
         plan.profile(False)
-        res["reuse"] = {"ms": reuse_ms, "launches": plan.launches(),
+        res["reuse"] = {"ms": reuse_ms, "launches": reuse_launches,
                         "stages": {k: round(v[0] / steps, 4) for k, v in rstages.items()}}
     if with_e2e:
         # End to end through the same C ABI call, from pinned host memory:

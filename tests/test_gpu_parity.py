@@ -266,3 +266,34 @@ def test_wait_that_runs_out_sets_timeout_and_context_recovers(w):
     again = B.httm_forward(plan, Q, K, V, workspace=ws)
     assert B.httm_get_device_status(plan, ws) == 0
     assert torch.equal(again, ref)
+
+
+@pytest.mark.parametrize("w", [MID, WORKLOADS["vggt_30f"], MID.with_(mode=HEAD_UNIFORM)],
+                         ids=["mid", "vggt_30f", "mid_head_uniform"])
+def test_forward_records_into_a_cuda_graph(w):
+    """A forward captured on a stream (its key branch forked onto the plan's
+    own stream and joined back by events) replays to the eager call's bits,
+    and re-plans from the data on each replay: new Q, K, V in the captured
+    buffers give the eager output of the new inputs."""
+    w, plan, _, (Q, K, V), _ = _case(w)
+    ws = plan.new_workspace()
+    eager = B.httm_forward(plan, Q, K, V, workspace=ws)       # first call binds the plan to the device
+    torch.cuda.synchronize()
+    ws_g = plan.new_workspace()
+    out_g = torch.empty_like(Q)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        B.httm_forward(plan, Q, K, V, out=out_g, workspace=ws_g)
+    g.replay()
+    torch.cuda.synchronize()
+    assert B.httm_get_device_status(plan, ws_g) == 0
+    assert torch.equal(out_g, eager)
+    Q2, K2, V2 = PL.inputs(w.with_(seed=w.seed + 1))
+    Q.copy_(Q2), K.copy_(K2), V.copy_(V2)
+    g.replay()
+    eager2 = B.httm_forward(plan, Q2, K2, V2, workspace=ws)
+    torch.cuda.synchronize()
+    assert B.httm_get_device_status(plan, ws_g) == 0
+    assert torch.equal(out_g, eager2)
+    assert not torch.equal(eager2, eager)
+    del g
