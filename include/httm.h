@@ -46,6 +46,7 @@ typedef enum {
   HTTM_ERR_CUDA = 6,             /* a CUDA runtime call failed */
   HTTM_ERR_TIMEOUT = 7,          /* device: a bounded wait ran out */
   HTTM_ERR_DEVICE_BOUNDS = 8,    /* device: an index was out of bounds / plan invalid */
+  HTTM_ERR_EXCHANGE = 9,         /* the caller's collective (httm_exchange) reported a failure */
 } httm_status;
 
 typedef enum { HTTM_BF16 = 0, HTTM_F32 = 1 } httm_dtype;
@@ -221,6 +222,56 @@ httm_status httm_forward_with_plan(httm_plan_t plan, const void* Q, const void* 
  */
 httm_status httm_forward_reuse(httm_plan_t plan, const void* Q, const void* K, const void* V,
                                void* out, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Head sharding (one layer over several GPUs).  Every step of the layer is
+ * per head except one: the outlier filter's budget, the top-d% of the
+ * deviations of ALL heads' queries (key design 3: the filter is global
+ * across heads, ties broken by the flat index h * N + n).  A layer of
+ * H = h * shards heads can therefore run as `shards` plans of h heads each,
+ * one per GPU, shard s holding heads [s * h, s * h + h) of Q, K, V and out,
+ * if the shards sum five small integer buffers between the filter's steps:
+ * the eligible-query count (4 B), the three radix histograms (8, 8 and
+ * 4 KB), and the per-shard counts of keys equal to the threshold (256 B).  The selection, and so the mask, is
+ * then exactly that of the unsharded layer.
+ *
+ * httm_exchange: the caller's collective.  allreduce_sum must sum `count`
+ * elements of `elem_bytes` bytes (4: uint32, 8: uint64) at the DEVICE
+ * address `buf` over all shards, in place, ordered on `stream` (work
+ * enqueued on `stream` after it returns sees the sums), e.g. an NCCL
+ * all-reduce; return 0 on success.  The library calls it from the thread
+ * that called httm_forward_sharded, the same number of times in the same
+ * order on every shard; `user` is passed through.
+ */
+typedef struct {
+  int32_t (*allreduce_sum)(void* buf, int64_t count, int32_t elem_bytes, void* stream, void* user);
+  void* user;
+} httm_exchange;
+
+/*
+ * httm_plan_shard: make `plan` (cfg.h = heads per shard) shard `shard` of
+ * `shards` of a head-sharded layer.  Changes the outlier budget to
+ * floor(d% * h * shards * N / 100) and so httm_workspace_bytes(); call it
+ * before the plan's first forward.  Errors: HTTM_ERR_ARG (shards < 1 or
+ * above 64, shard outside [0, shards), or the plan has already run);
+ * HTTM_ERR_UNSUPPORTED for HTTM_HEAD_UNIFORM with shards > 1 (its plan
+ * averages the cosines of all heads).
+ */
+httm_status httm_plan_shard(httm_plan_t plan, int32_t shard, int32_t shards);
+
+/*
+ * httm_forward_sharded: httm_forward (or, with a non-null dbg,
+ * httm_forward_debug) for one shard of a head-sharded layer, calling
+ * ex->allreduce_sum five times on `stream`.  ex may be NULL
+ * only for a single-shard plan.  A sharded plan runs only through this
+ * call: httm_forward, httm_forward_debug, httm_forward_with_plan and
+ * httm_forward_reuse return HTTM_ERR_ARG on it.  HTTM_ERR_EXCHANGE if a
+ * collective failed (the work already enqueued stays enqueued; the output
+ * is undefined).
+ */
+httm_status httm_forward_sharded(httm_plan_t plan, const void* Q, const void* K, const void* V, void* out,
+                                 void* workspace, size_t workspace_bytes, const httm_exchange* ex,
+                                 const httm_debug* dbg, void* stream);
 
 /*
  * httm_reorder: temporal reordering (key design 2).  inverse = 0: X in

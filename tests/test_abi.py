@@ -33,7 +33,7 @@ def test_library_exports_every_declared_symbol():
 
 def test_status_strings():
     lib = B.load_library()
-    for s in range(9):
+    for s in range(10):
         assert lib.httm_status_str(s).decode()
     assert lib.httm_status_str(99).decode() == "unknown status"
 
@@ -94,3 +94,32 @@ def test_contiguous_and_uniform_plans():
         blocks = O.block_list(_oracle_cfg(w.with_(mode=mode)))
         assert plan.info.n_blocks == len(blocks)
         assert plan.info.q_slots == sum(b.shape[0] - O.merge_count(b.shape[0], w.q_pct) for b in blocks)
+
+
+def test_head_shard_plan_sizes_and_errors():
+    """A shard of a head-sharded layer keeps its own heads' plan but the
+    whole layer's outlier budget (the filter is global across heads)."""
+    w = WORKLOADS["vggt_30f"]
+    full = B.httm_plan(B.LayerConfig.from_workload(w))
+    half = B.httm_plan(B.LayerConfig.from_workload(w, h=w.h // 2))
+    k_half = half.info.k_out_max
+    half.shard(1, 2)
+    assert half.info.k_out_max == w.out_pct * w.h * w.N // 100 == full.info.k_out_max
+    assert half.info.k_out_max > k_half
+    assert half.info.q_slots == full.info.q_slots and half.info.kv_slots == full.info.kv_slots
+    assert half.info.q_rows_alloc >= half.info.k_out_max
+    lib = B.load_library()
+    for shard, shards in ((2, 2), (-1, 2), (0, 0), (0, 65)):
+        assert lib.httm_plan_shard(half.handle, shard, shards) == 1      # HTTM_ERR_ARG
+    uni = B.httm_plan(B.LayerConfig.from_workload(w, h=w.h // 2, mode=B.HTTM_HEAD_UNIFORM))
+    assert lib.httm_plan_shard(uni.handle, 0, 2) == 2                     # HTTM_ERR_UNSUPPORTED
+    assert lib.httm_plan_shard(uni.handle, 0, 1) == 0
+    # a sharded plan runs only through httm_forward_sharded, with a collective;
+    # both are host checks made before any device call
+    fake = ctypes.c_void_p(1 << 20)
+    assert lib.httm_forward(half.handle, fake, fake, fake, fake, fake, 1 << 40, None) == 1
+    assert lib.httm_forward_reuse(half.handle, fake, fake, fake, fake, fake, 1 << 40, None) == 1
+    assert lib.httm_forward_sharded(half.handle, fake, fake, fake, fake, fake, 1 << 40, None, None, None) == 1
+    null_fn = B.httm_exchange()
+    assert lib.httm_forward_sharded(half.handle, fake, fake, fake, fake, fake, 1 << 40,
+                                    ctypes.byref(null_fn), None, None) == 1

@@ -9,12 +9,14 @@ from .binding import (  # noqa: F401
     HTTM_HEAD_UNIFORM,
     HTTM_HEADWISE_TEMPORAL,
     HttmError,
+    TorchExchange,
     LayerConfig,
     Plan,
     debug_buffers,
     httm_forward,
     httm_forward_debug,
     httm_forward_reuse,
+    httm_forward_sharded,
     httm_forward_with_plan,
     httm_get_device_status,
     httm_plan,

@@ -27,6 +27,7 @@ EXPORTS = (
     "httm_forward", "httm_forward_debug", "httm_forward_with_plan", "httm_forward_reuse", "httm_reorder",
     "httm_get_device_status", "httm_forward_launches", "httm_profile_enable", "httm_profile_read",
     "httm_select_outliers_noalloc", "httm_set_wait_budget", "httm_status_str",
+    "httm_plan_shard", "httm_forward_sharded",
 )
 STAGES = ("match", "merge", "outlier", "attention", "unmerge", "other")
 
@@ -57,6 +58,15 @@ class httm_debug(ctypes.Structure):
 
 class httm_merge_plan(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("q_best", "q_merged", "k_best", "k_merged", "outlier")]
+
+
+# int32_t (*allreduce_sum)(void* buf, int64_t count, int32_t elem_bytes, void* stream, void* user)
+EXCHANGE_FN = ctypes.CFUNCTYPE(ctypes.c_int32, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_void_p,
+                               ctypes.c_void_p)
+
+
+class httm_exchange(ctypes.Structure):
+    _fields_ = [("allreduce_sum", EXCHANGE_FN), ("user", ctypes.c_void_p)]
 
 
 _lib = None
@@ -93,11 +103,14 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.httm_select_outliers_noalloc.restype = ctypes.c_int
     lib.httm_set_wait_budget.argtypes = [P, ctypes.c_uint64]
     lib.httm_set_wait_budget.restype = ctypes.c_int
+    lib.httm_plan_shard.argtypes = [P, ctypes.c_int32, ctypes.c_int32]
+    lib.httm_forward_sharded.argtypes = [P, V, V, V, V, V, S, ctypes.POINTER(httm_exchange),
+                                         ctypes.POINTER(httm_debug), V]
     lib.httm_status_str.argtypes = [I]
     lib.httm_status_str.restype = ctypes.c_char_p
     for name in ("httm_plan", "httm_get_plan_info", "httm_forward", "httm_forward_debug",
                  "httm_forward_with_plan", "httm_forward_reuse", "httm_reorder", "httm_get_device_status",
-                 "httm_profile_enable", "httm_profile_read"):
+                 "httm_profile_enable", "httm_profile_read", "httm_plan_shard", "httm_forward_sharded"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -180,6 +193,17 @@ class Plan:
         if getattr(self, "handle", None) and _lib is not None:
             _lib.httm_plan_destroy(self.handle)
             self.handle = None
+
+    def shard(self, shard: int, shards: int) -> "Plan":
+        """Make this plan (cfg.h heads) shard `shard` of `shards` of a
+        head-sharded layer (httm_plan_shard); before its first forward."""
+        lib = load_library()
+        _check(lib.httm_plan_shard(self.handle, shard, shards), "httm_plan_shard")
+        info = httm_plan_info()
+        _check(lib.httm_get_plan_info(self.handle, ctypes.byref(info)), "httm_get_plan_info")
+        self.info = info
+        self.shard_index, self.shards = shard, shards
+        return self
 
     @property
     def workspace_bytes(self) -> int:
@@ -338,3 +362,63 @@ def httm_select_outliers_noalloc(dev, eligible, outlier_pct: int, mask=None, n_o
                                                        _ptr(n_out), _stream(stream)),
            "httm_select_outliers_noalloc")
     return mask, n_out
+
+
+def exchange_view(ws: torch.Tensor, buf, count: int, elem_bytes: int) -> torch.Tensor:
+    """The int32 / int64 view of `ws` (a uint8 workspace tensor) at the
+    address `buf` that an httm_exchange call names; raises if it is not
+    inside the workspace or not aligned."""
+    if ws is None or not buf:
+        raise ValueError("no workspace for this exchange")
+    off, n = int(buf) - ws.data_ptr(), int(count) * int(elem_bytes)
+    if off < 0 or off + n > ws.numel() or elem_bytes not in (4, 8) or off % elem_bytes:
+        raise ValueError("exchange buffer outside the workspace")
+    return ws[off: off + n].view(torch.int32 if elem_bytes == 4 else torch.int64)
+
+
+class TorchExchange:
+    """``httm_exchange`` over torch.distributed: every sum the library asks
+    for is ``dist.all_reduce`` of a view of the call's workspace (the library
+    only sums buffers inside it), issued on the library's stream -- NCCL for
+    CUDA workspaces, gloo for CPU tensors.  One object per thread of calls."""
+
+    def __init__(self, group=None):
+        self.group = group
+        self.workspace = None
+        self.calls = 0
+        self._fn = EXCHANGE_FN(self._allreduce_sum)
+        self.c = httm_exchange(self._fn, None)
+
+    def _allreduce_sum(self, buf, count, elem_bytes, stream, user) -> int:
+        import torch.distributed as dist
+        try:
+            t = exchange_view(self.workspace, buf, count, elem_bytes)
+            if t.is_cuda:
+                s = torch.cuda.ExternalStream(stream, device=t.device) if stream else \
+                    torch.cuda.default_stream(t.device)
+                with torch.cuda.stream(s):
+                    dist.all_reduce(t, group=self.group)
+            else:
+                dist.all_reduce(t, group=self.group)
+            self.calls += 1
+            return 0
+        except Exception:   # reported to the library, which returns HTTM_ERR_EXCHANGE
+            return 1
+
+
+def httm_forward_sharded(plan: Plan, Q, K, V, exchange, out=None, workspace=None, dbg: dict | None = None,
+                         stream=None):
+    """One shard of a head-sharded layer (Q, K, V: this shard's heads).
+    ``exchange`` has a ``c`` (httm_exchange) and a ``workspace`` attribute,
+    set here to the call's workspace (:class:`TorchExchange`), or is None
+    for a single-shard plan."""
+    out, workspace = _prep(plan, Q, K, V, out, workspace)
+    ex = None
+    if exchange is not None:
+        exchange.workspace = workspace
+        ex = ctypes.byref(exchange.c)
+    d = ctypes.byref(_debug_struct(dbg)) if dbg is not None else None
+    _check(load_library().httm_forward_sharded(plan.handle, _ptr(Q), _ptr(K), _ptr(V), _ptr(out),
+                                               _ptr(workspace), workspace.numel(), ex, d, _stream(stream)),
+           "httm_forward_sharded")
+    return out

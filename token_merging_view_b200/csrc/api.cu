@@ -99,7 +99,7 @@ Workspace layout(const Dims& d, bool fp32) {
     return o;
   };
   w.state = take(sizeof(DevState));
-  w.hist = take(3ull * kHistBins * 4);
+  w.hist = take((3ull * kHistBins + kMaxShards) * 4);
   w.chunk = take((size_t)d.h * d.nchunk_per_head * 16);
   w.n_out = take((size_t)d.h * 4);
   w.out_base = take((size_t)d.h * 4);
@@ -162,6 +162,18 @@ Buffers resolve(const Workspace& w, void* base) {
   b.o_tilde = p + w.o_tilde;
   b.attn_part = reinterpret_cast<float*>(p + w.attn_part);
   return b;
+}
+
+// The outlier budget of the whole layer (all shards' heads) and the
+// outlier rows, work items and workspace it needs: one shard may receive
+// every outlier of the layer.
+void size_outliers(Dims& d, int outlier_pct) {
+  const long long heads = (long long)d.h * d.shards;
+  d.k_out_max = ((long long)outlier_pct * heads * d.N) / 100;
+  d.out_base = (long long)align_up((size_t)d.h * d.q_slots, kAttnRows);
+  d.q_rows_alloc = d.out_base + d.k_out_max + (long long)kAttnRows * (d.h + 1);
+  d.max_items = (int32_t)(d.h * ((d.q_slots + kAttnRows - 1) / kAttnRows) + (d.k_out_max + kAttnRows - 1) / kAttnRows +
+                          d.h);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -235,10 +247,38 @@ httm_status attention(const httm_plan_s* plan, const void* q, const void* k, con
   return e == cudaSuccess ? HTTM_OK : HTTM_ERR_CUDA;
 }
 
+// The outlier filter (without its restore).  With a collective (a
+// head-sharded layer), the shards sum the eligible count and the first
+// histogram (both built by the query gather), each later histogram, and the
+// per-shard counts of keys equal to the threshold, between the steps.
+httm_status outlier_stage(const Dims& dims, bool fp32, const void* Q, bool mask_inj, const Buffers& buf,
+                          cudaStream_t s, const httm_exchange* ex, int* launches) {
+  if (!ex) {
+    const cudaError_t e = launch_outlier(dims, fp32, Q, mask_inj, buf, s);
+    *launches += mask_inj ? 3 : 5;  // two histogram passes, count, scan, emit
+    return e == cudaSuccess ? HTTM_OK : HTTM_ERR_CUDA;
+  }
+  auto sum = [&](void* p, int64_t n, int32_t eb) { return ex->allreduce_sum(p, n, eb, s, ex->user) == 0; };
+  if (!sum(&buf.state->n_eligible, 1, 4) || !sum(buf.hist, kHistBins, 4)) return HTTM_ERR_EXCHANGE;
+  for (int pass = 2; pass <= 3; ++pass) {
+    if (launch_outlier_pass(dims, buf, pass, s) != cudaSuccess) return HTTM_ERR_CUDA;
+    ++*launches;
+    if (!sum(buf.hist + (pass - 1) * kHistBins, pass == 2 ? kHistBins : 1024, 4)) return HTTM_ERR_EXCHANGE;
+  }
+  if (launch_outlier_count(dims, false, buf, s) != cudaSuccess) return HTTM_ERR_CUDA;
+  ++*launches;
+  if (!sum(buf.hist + 3 * kHistBins, kMaxShards, 4)) return HTTM_ERR_EXCHANGE;
+  if (launch_outlier_emit(dims, fp32, Q, false, buf, s) != cudaSuccess) return HTTM_ERR_CUDA;
+  *launches += 2;  // scan, emit
+  return HTTM_OK;
+}
+
 httm_status forward_impl(httm_plan_s* plan, const void* Q, const void* K, const void* V, void* out, void* ws,
                          size_t ws_bytes, const httm_merge_plan* inj, const httm_debug* dbg, void* stream,
-                         bool reuse = false) {
+                         bool reuse = false, bool sharded_call = false, const httm_exchange* ex = nullptr) {
   if (!plan || !Q || !K || !V || !out || !ws) return HTTM_ERR_ARG;
+  if (plan->dims.shards > 1 && (!sharded_call || !ex)) return HTTM_ERR_ARG;
+  if (ex && !ex->allreduce_sum) return HTTM_ERR_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(out)) return HTTM_ERR_ALIGN;
   if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return HTTM_ERR_ALIGN;
   if (reuse && (inj || plan->dims.mode == HTTM_DENSE)) return HTTM_ERR_ARG;
@@ -300,8 +340,7 @@ httm_status forward_impl(httm_plan_s* plan, const void* Q, const void* K, const 
     HTTM_LAUNCH(launch_merge(dims, fp32, plan->blocks_d, plan_inj, reuse, Q, K, V, buf, dd, s, 1));
     HTTM_LAUNCH(launch_merge(dims, fp32, plan->blocks_d, plan_inj, reuse, Q, K, V, buf, dd, s2, 2));
     if (!reuse) launches += 2;  // the two planning launches
-    HTTM_LAUNCH(launch_outlier(dims, fp32, Q, mask_inj, buf, s));
-    launches += mask_inj ? 2 : 4;
+    if ((st = outlier_stage(dims, fp32, Q, mask_inj, buf, s, ex, &launches)) != HTTM_OK) return st;
     HTTM_LAUNCH(launch_restore(dims, fp32, plan->blocks_d, Q, buf, dd, s));
     if (cudaEventRecord(plan->ev_join, s2) != cudaSuccess || cudaStreamWaitEvent(s, plan->ev_join, 0) != cudaSuccess)
       return HTTM_ERR_CUDA;
@@ -329,8 +368,7 @@ httm_status forward_impl(httm_plan_s* plan, const void* Q, const void* K, const 
   }
   {
     StageTimer t(plan, s, HTTM_STAGE_OUTLIER, mask_inj ? 4 : 6);
-    HTTM_LAUNCH(launch_outlier(dims, fp32, Q, mask_inj, buf, s));
-    launches += mask_inj ? 2 : 4;  // count, scan, emit, plus two histogram passes
+    if ((st = outlier_stage(dims, fp32, Q, mask_inj, buf, s, ex, &launches)) != HTTM_OK) return st;
     HTTM_LAUNCH(launch_restore(dims, fp32, plan->blocks_d, Q, buf, dd, s));
   }
   {
@@ -365,6 +403,7 @@ const char* httm_status_str(httm_status s) {
     case HTTM_ERR_CUDA: return "CUDA runtime error";
     case HTTM_ERR_TIMEOUT: return "device wait timed out";
     case HTTM_ERR_DEVICE_BOUNDS: return "device bounds / plan check failed";
+    case HTTM_ERR_EXCHANGE: return "the caller's collective failed";
   }
   return "unknown status";
 }
@@ -407,6 +446,8 @@ httm_status httm_plan(const httm_cfg* cfg, httm_plan_t* out) {
   d.plan_id = next_id.fetch_add(1);
   if (d.plan_id == 0) d.plan_id = next_id.fetch_add(1);
   d.wait_budget_ns = 2000000000ull;
+  d.shard = 0;
+  d.shards = 1;
   d.nchunk_per_head = (int32_t)((N + kChunk - 1) / kChunk);
   if (c.mode == HTTM_DENSE) {
     d.max_items = (int32_t)(c.h * ((N + kAttnRows - 1) / kAttnRows));
@@ -470,10 +511,7 @@ httm_status httm_plan(const httm_cfg* cfg, httm_plan_t* out) {
     d.k_src = ks;
     d.q_slots = qsl;
     d.k_slots = ksl;
-    d.k_out_max = ((long long)c.outlier_pct * c.h * N) / 100;
-    d.out_base = (long long)align_up((size_t)c.h * qsl, kAttnRows);
-    d.q_rows_alloc = d.out_base + d.k_out_max + (long long)kAttnRows * (c.h + 1);
-    d.max_items = (int32_t)(c.h * ((qsl + kAttnRows - 1) / kAttnRows) + (d.k_out_max + kAttnRows - 1) / kAttnRows + c.h);
+    size_outliers(d, c.outlier_pct);
     // matching work: 128-source tiles of every (tensor, block), costliest first
     std::vector<int4> items;
     for (int t = 0; t < 2; ++t)
@@ -582,6 +620,28 @@ httm_status httm_forward_with_plan(httm_plan_t plan, const void* Q, const void* 
 httm_status httm_forward_reuse(httm_plan_t plan, const void* Q, const void* K, const void* V, void* out,
                                void* workspace, size_t workspace_bytes, void* stream) {
   return forward_impl(plan, Q, K, V, out, workspace, workspace_bytes, nullptr, nullptr, stream, true);
+}
+
+httm_status httm_plan_shard(httm_plan_t plan, int32_t shard, int32_t shards) {
+  if (!plan || shards < 1 || shards > kMaxShards || shard < 0 || shard >= shards || plan->device >= 0)
+    return HTTM_ERR_ARG;
+  if (plan->dims.mode == HTTM_HEAD_UNIFORM && shards > 1) return HTTM_ERR_UNSUPPORTED;
+  Dims d = plan->dims;
+  d.shard = shard;
+  d.shards = shards;
+  if (d.mode != HTTM_DENSE) {
+    size_outliers(d, plan->cfg.outlier_pct);
+    if (d.k_out_max > (1ll << 31) - 1 || d.q_rows_alloc > (1ll << 31) - 1) return HTTM_ERR_UNSUPPORTED;
+  }
+  plan->dims = d;
+  plan->ws = layout(d, plan->fp32);
+  return HTTM_OK;
+}
+
+httm_status httm_forward_sharded(httm_plan_t plan, const void* Q, const void* K, const void* V, void* out,
+                                 void* workspace, size_t workspace_bytes, const httm_exchange* ex,
+                                 const httm_debug* dbg, void* stream) {
+  return forward_impl(plan, Q, K, V, out, workspace, workspace_bytes, nullptr, dbg, stream, false, true, ex);
 }
 
 httm_status httm_reorder(httm_plan_t plan, const void* X, void* Xb, int inverse, void* stream) {

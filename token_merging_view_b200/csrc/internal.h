@@ -39,10 +39,12 @@ struct Dims {
   float scale;
   uint32_t plan_id;              // stamps a workspace whose member lists this plan wrote
   uint64_t wait_budget_ns;       // bound of a device wait (httm_set_wait_budget; default 2 s)
+  int32_t shard, shards;         // head sharding: this shard holds heads [shard h, shard h + h) of h shards
 };
 
 constexpr int kChunk = 4096;       // keys per chunk of the outlier compaction
 constexpr int kHistBins = 2048;    // radix digit of the outlier select (11 bits)
+constexpr int kMaxShards = 64;     // head shards of one layer (httm_plan_shard)
 constexpr int kAttnRows = 256;     // query rows per attention work item (two 128-row tiles)
 constexpr int kMaxAttnParts = 256; // partial results of the last wave's split items (<= one per SM)
 constexpr int kAttnPartStride = 68; // floats per partial row: O (64), row sum, max in use, 2 unused (16-byte rows)
@@ -76,7 +78,7 @@ struct Debug;  // mirrors httm_debug
 // Pointers into one forward's workspace, resolved on the host.
 struct Buffers {
   DevState* state;
-  uint32_t* hist;          // [3][kHistBins]
+  uint32_t* hist;          // [3][kHistBins], then [kMaxShards]: keys equal to the threshold per shard
   uint32_t* chunk;         // [nchunk][4]: gt, eq, take, out_before
   int32_t* n_out;          // [h]
   int32_t* out_base;       // [h]

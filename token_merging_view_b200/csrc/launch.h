@@ -48,6 +48,14 @@ cudaError_t launch_merge(const Dims& dims, bool fp32, const BlockDesc* blocks, b
 
 cudaError_t launch_outlier(const Dims& dims, bool fp32, const void* Q, bool mask_injected,
                            const Buffers& buf, cudaStream_t s);
+// The same filter in steps, for a head-sharded layer whose shards sum the
+// eligible count and each radix histogram between steps (and, after the
+// count step, the per-shard counts of keys equal to the threshold):
+// histogram pass 2 or 3, then count, then scan + emit.
+cudaError_t launch_outlier_pass(const Dims& dims, const Buffers& buf, int pass, cudaStream_t s);
+cudaError_t launch_outlier_count(const Dims& dims, bool mask_injected, const Buffers& buf, cudaStream_t s);
+cudaError_t launch_outlier_emit(const Dims& dims, bool fp32, const void* Q, bool mask_injected,
+                                const Buffers& buf, cudaStream_t s);
 
 cudaError_t launch_restore(const Dims& dims, bool fp32, const BlockDesc* blocks, const void* Q,
                            const Buffers& buf, const Debug& dbg, cudaStream_t s);

@@ -829,7 +829,7 @@ __global__ void export_kernel(Dims dims, const BlockDesc* __restrict__ blocks, B
 }
 
 __global__ void zero_state_kernel(Buffers buf, int keep_stamp, unsigned long long wait_ns) {
-  for (int i = threadIdx.x; i < 3 * kHistBins; i += blockDim.x) buf.hist[i] = 0u;
+  for (int i = threadIdx.x; i < 3 * kHistBins + kMaxShards; i += blockDim.x) buf.hist[i] = 0u;
   if (threadIdx.x == 0) {
     if (!keep_stamp) buf.state->plan_stamp = 0u;   // rewritten once this call's planning has succeeded
     buf.state->status = 0u;

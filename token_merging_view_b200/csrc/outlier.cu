@@ -14,6 +14,12 @@
 // T in flat-index order, found with chunk counts and a scan.  Every step is
 // its own launch (no grid-wide barrier, no spin wait), and every count is an
 // integer, so the mask is deterministic.
+//
+// Head sharding: the histograms count this shard's heads only; the caller's
+// collective sums them over the shards between the steps, so every shard
+// finds the same T and budget.  Keys equal to T are taken in flat-index
+// order over the whole layer: each shard counts its own, and the shards
+// before it (lower heads) take theirs first.
 #include <algorithm>
 
 #include "common.cuh"
@@ -130,6 +136,7 @@ __global__ void __launch_bounds__(1024) out_count_kernel(Dims dims, Buffers buf,
   if (threadIdx.x == 0) {
     buf.chunk[4 * c + 0] = gt;
     buf.chunk[4 * c + 1] = eq;
+    if (eq) atomicAdd(&buf.hist[3 * kHistBins + dims.shard], eq);   // this shard's keys equal to T
     if (c == 0) {
       buf.state->sel[0] = T;
       buf.state->sel[1] = need;
@@ -147,7 +154,13 @@ __global__ void __launch_bounds__(1024) out_scan_kernel(Dims dims, Buffers buf) 
   const int tid = threadIdx.x;
   const int cph = dims.nchunk_per_head;
   const int nchunk = dims.h * cph;
-  const uint32_t need = buf.state->sel[1];
+  // Equal keys are taken in flat-index order over all heads of the layer:
+  // the shards before this one (lower heads) take theirs first.
+  const uint32_t* eq_shard = buf.hist + 3 * kHistBins;
+  uint32_t before = 0;
+  for (int r = 0; r < dims.shard; ++r) before += eq_shard[r];
+  const uint32_t need_all = buf.state->sel[1];
+  const uint32_t need = need_all > before ? min(need_all - before, eq_shard[dims.shard]) : 0u;
   uint32_t carry = 0;
   for (int base = 0; base < nchunk; base += blockDim.x) {
     const int c = base + tid;
@@ -302,16 +315,32 @@ __global__ void dense_items_kernel(Dims dims, Buffers buf) {
 
 }  // namespace
 
-cudaError_t launch_outlier(const Dims& dims, bool fp32, const void* Q, bool mask_injected,
-                           const Buffers& buf, cudaStream_t s) {
+cudaError_t launch_outlier_pass(const Dims& dims, const Buffers& buf, int pass, cudaStream_t s) {
   const size_t total = (size_t)dims.h * dims.N;
   const int hgrid = (int)std::max<size_t>(1, std::min<size_t>((total + 4095) / 4096, 148 * 2));
+  hist_pass_kernel<<<hgrid, 1024, 0, s>>>(dims, buf, pass);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_outlier_count(const Dims& dims, bool mask_injected, const Buffers& buf, cudaStream_t s) {
+  out_count_kernel<<<dims.h * dims.nchunk_per_head, 1024, 0, s>>>(dims, buf, mask_injected ? 1 : 0);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_outlier(const Dims& dims, bool fp32, const void* Q, bool mask_injected,
+                           const Buffers& buf, cudaStream_t s) {
+  cudaError_t e;
   if (!mask_injected) {
-    hist_pass_kernel<<<hgrid, 1024, 0, s>>>(dims, buf, 2);
-    hist_pass_kernel<<<hgrid, 1024, 0, s>>>(dims, buf, 3);
+    if ((e = launch_outlier_pass(dims, buf, 2, s)) != cudaSuccess) return e;
+    if ((e = launch_outlier_pass(dims, buf, 3, s)) != cudaSuccess) return e;
   }
+  if ((e = launch_outlier_count(dims, mask_injected, buf, s)) != cudaSuccess) return e;
+  return launch_outlier_emit(dims, fp32, Q, mask_injected, buf, s);
+}
+
+cudaError_t launch_outlier_emit(const Dims& dims, bool fp32, const void* Q, bool mask_injected,
+                                const Buffers& buf, cudaStream_t s) {
   const int nchunk = dims.h * dims.nchunk_per_head;
-  out_count_kernel<<<nchunk, 1024, 0, s>>>(dims, buf, mask_injected ? 1 : 0);
   out_scan_kernel<<<1, 1024, 0, s>>>(dims, buf);
   const int mi = mask_injected ? 1 : 0;
   if (fp32) {
