@@ -262,7 +262,7 @@ httm_status httm_plan_shard(httm_plan_t plan, int32_t shard, int32_t shards);
 /*
  * httm_forward_sharded: httm_forward (or, with a non-null dbg,
  * httm_forward_debug) for one shard of a head-sharded layer, calling
- * ex->allreduce_sum five times on `stream`.  ex may be NULL
+ * ex->allreduce_sum five times on `stream` (never in HTTM_DENSE mode).  ex may be NULL
  * only for a single-shard plan.  A sharded plan runs only through this
  * call: httm_forward, httm_forward_debug, httm_forward_with_plan and
  * httm_forward_reuse return HTTM_ERR_ARG on it.  HTTM_ERR_EXCHANGE if a
