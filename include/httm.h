@@ -25,6 +25,10 @@
  *    starts; httm_get_device_status() reads it.
  *  - Nothing throws across this boundary.  The library allocates no device
  *    memory except the small block table owned by a plan.
+ *  - A plan is not thread-safe: calls on one plan from several host threads
+ *    must not overlap (the caller serialises them, or gives each thread a
+ *    plan of its own; plans are cheap).  Calls on different plans may run
+ *    concurrently from any threads.
  */
 #ifndef HTTM_H_
 #define HTTM_H_
@@ -145,8 +149,8 @@ size_t httm_workspace_bytes(httm_plan_t plan);
  * key branch (matching, planning and gathering K/V) runs on the plan's own
  * stream, forked from `stream` by an event at the call's start and joined
  * back before attention, so the call stays ordered on `stream` and records
- * into a CUDA graph captured on it; calls on one plan from several streams
- * at once share that stream, which only serialises their key branches.
+ * into a CUDA graph captured on it; calls on one plan enqueued on several
+ * streams share that stream, which only serialises their key branches.
  */
 httm_status httm_forward(httm_plan_t plan, const void* Q, const void* K, const void* V,
                          void* out, void* workspace, size_t workspace_bytes, void* stream);
