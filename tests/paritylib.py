@@ -151,6 +151,33 @@ def sample_out_error(res: O.OracleResult, out_g: np.ndarray, cfg: O.OracleConfig
     return max(errs), np.sqrt(nums / dens)
 
 
+def sample_slot_error(res: O.OracleResult, out_g, cfg: O.OracleConfig, slots_per_head: int, seed: int = 0):
+    """Oracle attention for a seeded sample of the live query slots of each
+    head (all of them if the head has fewer), compared at every token whose
+    output comes from a sampled slot, so the unmerge's fan-out is checked as
+    well.  out_g: the GPU output, a torch tensor (any device) or an array,
+    [h, N, d].  Returns (max abs error, relative L2 error, slots compared)."""
+    rng = np.random.default_rng(seed)
+    h = res.restore.slot_final.shape[0]
+    errs, nums, dens, n_slots = [], 0.0, 0.0, 0
+    for hh in range(h):
+        sf = res.restore.slot_final[hh]
+        live = np.unique(sf)                  # drained slots are read by no token
+        chosen = live if live.size <= slots_per_head else np.sort(rng.choice(live, slots_per_head, replace=False))
+        toks = np.nonzero(np.isin(sf, chosen))[0]
+        inv = np.searchsorted(chosen, sf[toks])
+        o = O.attention(res.restore.q_tilde[hh][chosen], res.k_means[hh], res.v_means[hh], cfg.softmax_scale)[inv]
+        if isinstance(out_g, torch.Tensor):
+            g = out_g[hh][torch.from_numpy(toks).to(out_g.device)].double().cpu().numpy()
+        else:
+            g = np.asarray(out_g[hh, toks], dtype=np.float64)
+        errs.append(np.abs(g - o).max())
+        nums += float(((g - o) ** 2).sum())
+        dens += float((o ** 2).sum())
+        n_slots += chosen.size
+    return max(errs), np.sqrt(nums / dens), n_slots
+
+
 def run(plan: B.Plan, Q, K, V, injected=None, debug=True):
     dbg = B.debug_buffers(plan) if debug else None
     ws = plan.new_workspace()

@@ -28,7 +28,7 @@ def _case(w: Workload, **kw):
     return w, plan, cfg, (Q, K, V), tuple(PL.to64(t) for t in (Q, K, V))
 
 
-def _full_check(w: Workload, tokens_per_head: int = 1 << 30, max_excused_frac: float = 1e-3):
+def _full_check(w: Workload, slots_per_head: int = 1 << 30, max_excused_frac: float = 1e-3):
     w, plan, cfg, (Q, K, V), (q, k, v) = _case(w)
     res = O.forward_plan(cfg, q, k, v)
     # 1. the layer's own plan
@@ -64,10 +64,10 @@ def _full_check(w: Workload, tokens_per_head: int = 1 << 30, max_excused_frac: f
     assert np.array_equal(B.workspace_view(plan, ws3, "n_out").cpu().numpy(), res.restore.n_out)
     assert np.array_equal(dbg3["q_slot"], res.restore.slot_final)
     assert np.array_equal(dbg3["outlier"].astype(bool), res.mask)
-    mx, rl2 = PL.sample_out_error(res, PL.to64(out3), cfg, tokens_per_head)
+    mx, rl2, _ = PL.sample_slot_error(res, out3, cfg, slots_per_head)
     assert mx <= PL.OUT_MAX_ABS and rl2 <= PL.OUT_REL_L2, (mx, rl2)
     # the layer's own end-to-end output stays within the same bound
-    mx, rl2 = PL.sample_out_error(res, PL.to64(out), cfg, min(tokens_per_head, 256), seed=1)
+    mx, rl2, _ = PL.sample_slot_error(res, out, cfg, min(slots_per_head, 256), seed=1)
     return ex, n_mask_ex, (mx, rl2)
 
 
@@ -95,19 +95,19 @@ def test_mid_layer_edge_cases(kw):
 
 
 def test_vggt_30f_layer():
-    _full_check(WORKLOADS["vggt_30f"], tokens_per_head=512)
+    _full_check(WORKLOADS["vggt_30f"], slots_per_head=4096)
 
 
 @pytest.mark.slow
 def test_vggt_100f_layer_sampled():
-    _full_check(WORKLOADS["vggt_100f"], tokens_per_head=128)
+    _full_check(WORKLOADS["vggt_100f"], slots_per_head=4096)
 
 
 @pytest.mark.slow
 def test_vggt_500f_layer_sampled():
     """The 500-frame layer (684,500 tokens, queries with destinations every
     8th token and 85% merged) in the launch configuration bench.py times."""
-    _full_check(WORKLOADS["vggt_500f"], tokens_per_head=48)
+    _full_check(WORKLOADS["vggt_500f"], slots_per_head=4096)
 
 
 def test_reorder_matches_oracle():
@@ -240,7 +240,7 @@ def test_vggt_30f_head_uniform_plan():
     """The head-uniform plan at the 30-frame layer's shape (16 heads, blocks
     of 3840 / 2670 tokens) from the tensor-core matcher: the plan against the
     oracle's, and the output on the oracle's plan and mask."""
-    _full_check(WORKLOADS["vggt_30f"].with_(mode=HEAD_UNIFORM), tokens_per_head=256)
+    _full_check(WORKLOADS["vggt_30f"].with_(mode=HEAD_UNIFORM), slots_per_head=4096)
 
 
 @pytest.mark.parametrize("kw", [dict(d=16), dict(fp32=True, T=3, h=2)], ids=["bf16_d16", "fp32_d64"])
