@@ -26,36 +26,6 @@ namespace {
 constexpr int kMergeThreads = 256;
 static_assert(kMergeThreads == 256, "the planning kernel clears and selects 256 radix bins, one per thread");
 
-// A [D]-row spread over one warp: lane l owns elements [l*E, l*E + E).
-template <class T, int D>
-struct WarpRow {
-  static constexpr int E = D >= 32 ? D / 32 : 1;
-  __device__ static bool owns(int lane) { return lane * E < D; }
-  __device__ static void load(const T* row, int lane, float (&v)[E]) {
-#pragma unroll
-    for (int e = 0; e < E; ++e) v[e] = owns(lane) ? to_f(row[lane * E + e]) : 0.f;
-  }
-  __device__ static void store(T* row, int lane, const float (&v)[E]) {
-    if (!owns(lane)) return;
-#pragma unroll
-    for (int e = 0; e < E; ++e) row[lane * E + e] = from_f<T>(v[e]);
-  }
-};
-
-template <>
-struct WarpRow<__nv_bfloat16, 64> {
-  static constexpr int E = 2;
-  __device__ static bool owns(int) { return true; }
-  __device__ static void load(const __nv_bfloat16* row, int lane, float (&v)[2]) {
-    const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(row) + lane);
-    v[0] = __uint_as_float(w << 16);
-    v[1] = __uint_as_float(w & 0xffff0000u);
-  }
-  __device__ static void store(__nv_bfloat16* row, int lane, const float (&v)[2]) {
-    reinterpret_cast<__nv_bfloat162*>(row)[lane] = __floats2bfloat162_rn(v[0], v[1]);
-  }
-};
-
 // A row as 16-byte chunks spread over a warp: CPR chunks per row, RPI rows
 // per warp-wide access, EPC elements per chunk.
 template <class T, int D>
