@@ -104,7 +104,8 @@ typedef struct {
   int32_t n_blocks;       /* merge blocks per head */
   int32_t q_slots;        /* regular query slots R_q = sum_b (n_b - r_b^Q) */
   int32_t kv_slots;       /* key/value slots L_k = sum_b (n_b - r_b^KV) */
-  int64_t k_out_max;      /* floor(outlier_pct * h * N / 100): outlier budget, all heads */
+  int64_t k_out_max;      /* floor(outlier_pct * H * N / 100): outlier budget of all H heads of
+                             the layer (H = h, or h * shards after httm_plan_shard) */
   int64_t q_rows_alloc;   /* rows of the shortened-query buffer (all heads, padded) */
   int64_t ws_q_tilde;     /* workspace byte offsets of the shortened tensors: */
   int64_t ws_k_tilde;     /*   Q~ rows [q_rows_alloc, d] (regular slots of head hh at */
