@@ -1,8 +1,10 @@
 // Allocation-free variant of the global outlier selection.
 //
-// Same selection as the forward's filter stage: among the queries flagged
-// eligible, the k = min(floor(pct * h * N / 100), #eligible) with the
-// largest deviation, ties by ascending flat index h * N + n.  It differs in
+// Same selection as the forward's filter stage ("HTTM: Head-wise Temporal
+// Token Merging for Faster VGGT", key design 3, the cross-head adaptive
+// outlier filter): among the queries flagged eligible, the
+// k = min(floor(pct * h * N / 100), #eligible) with the largest deviation,
+// ties by ascending flat index h * N + n.  It differs in
 // where its scratch (radix histograms, per-chunk counts, counters) lives:
 // not in a caller workspace but in g_select_scratch below, a file-scope
 // device array of fixed size, so a call allocates nothing at all.
