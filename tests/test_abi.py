@@ -123,3 +123,21 @@ def test_head_shard_plan_sizes_and_errors():
     null_fn = B.httm_exchange()
     assert lib.httm_forward_sharded(half.handle, fake, fake, fake, fake, fake, 1 << 40,
                                     ctypes.byref(null_fn), None, None) == 1
+
+
+def test_binding_rejects_bad_tensors_before_any_device_call():
+    """The binding only marshals: host tensors, a wrong dtype or a strided
+    view are refused in Python, so no pointer of the wrong kind reaches the
+    library (which would treat it as device memory)."""
+    import torch
+    w = WORKLOADS["tiny_4f_8x8"]
+    plan = B.httm_plan(B.LayerConfig.from_workload(w))
+    shape = (w.h, w.N, w.d)
+    Q = torch.zeros(shape, dtype=torch.float32)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        B.httm_forward(plan, Q, Q, Q, out=torch.empty_like(Q), workspace=torch.empty(plan.workspace_bytes,
+                                                                                      dtype=torch.uint8))
+    with pytest.raises(ValueError, match="contiguous"):
+        B.httm_forward(plan, Q.to(torch.bfloat16), Q, Q)
+    with pytest.raises(ValueError, match="contiguous"):
+        B.httm_forward(plan, Q.transpose(1, 2).contiguous().transpose(1, 2), Q, Q)
