@@ -83,3 +83,52 @@ def softmax_attention_row(q, Ks, Vs, scale):
     w = [math.exp(v - m) for v in z]
     s = sum(w)
     return [sum(w[j] * Vs[j][c] for j in range(len(Ks))) / s for c in range(len(Vs[0]))]
+
+
+def partition_roles(score, grid, ga_pct):
+    """LiteVGGT's token classes by loops: score is a list (frames) of lists
+    (raster patches).  Returns a list of lists of 'ga' / 'dst' / 'src'."""
+    P = grid * grid
+    k = ga_pct * P // 100
+    out = []
+    for t, row in enumerate(score):
+        by_importance = sorted(range(P), key=lambda p: (-row[p], p))
+        ga = set(by_importance[:k])
+        roles = ['ga' if p in ga else None for p in range(P)]
+        if t == 0:
+            roles = ['ga' if p in ga else 'dst' for p in range(P)]
+            out.append(roles)
+            continue
+        for cy in range(0, grid, 2):
+            for cx in range(0, grid, 2):
+                members = [y * grid + x for y in range(cy, min(cy + 2, grid))
+                           for x in range(cx, min(cx + 2, grid))]
+                free = [p for p in members if p not in ga]
+                if not free:
+                    continue
+                anchor = min(free, key=lambda p: (row[p], p))
+                for p in free:
+                    roles[p] = 'dst' if p == anchor else 'src'
+        out.append(roles)
+    return out
+
+
+def match_block_roles(rows, roles):
+    """rows, roles: in-block order.  Every 'src' joins its most similar 'dst'
+    (ties: the lowest in-block index); 'ga' tokens and the sources of a block
+    without destinations stay alone.  Returns the member lists: one per dst
+    in ascending order, then one per singleton in ascending order."""
+    dst = [i for i, r in enumerate(roles) if r == 'dst']
+    join = {}
+    for s, r in enumerate(roles):
+        if r != 'src' or not dst:
+            continue
+        bi, bv = None, None
+        for t in dst:
+            c = cos(rows[s], rows[t])
+            if bv is None or c > bv:
+                bi, bv = t, c
+        join[s] = bi
+    groups_ = [[t] + [s for s in sorted(join) if join[s] == t] for t in dst]
+    groups_ += [[i] for i, r in enumerate(roles) if r != 'dst' and i not in join]
+    return groups_

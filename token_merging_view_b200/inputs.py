@@ -93,3 +93,17 @@ def make_qkv(
         out.append(x.reshape(h, T * P, d).to(dtype).contiguous())
         del z, f, field, e, x
     return tuple(out)
+
+
+def make_score(*, T: int, grid: int, seed: int, blur_sigma: float = 1.5, blur_radius: int = 6,
+               device: str | torch.device = "cpu") -> torch.Tensor:
+    """A seeded stand-in for a per-token importance map, fp32 [T, grid*grid]:
+    per frame an N(0, 1) field on the patch grid, blurred like the Q/K/V
+    fields (so neighbouring patches score alike, as edges and flat regions
+    do in an image).  Holds no part of any method: inputs only."""
+    device = torch.device(device)
+    gen = torch.Generator(device=device).manual_seed(seed)
+    z = torch.randn((T, grid, grid, 1), generator=gen, device=device, dtype=torch.float64)
+    radius = min(blur_radius, grid - 1)                 # a mirror pad needs radius < grid
+    f = _blur_field(z, _gauss_weights(blur_sigma, radius).to(device)) if radius > 0 else z
+    return f.reshape(T, grid * grid).float()
