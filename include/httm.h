@@ -349,8 +349,11 @@ httm_status httm_profile_read(httm_plan_t plan, float* ms, int32_t* launches);
  * consecutive calls are independent -- but calls that overlap on the GPU
  * (different streams, or different host threads, at the same time) race and
  * give undefined results.  The first call on each device looks up the
- * array's device address (a host-side set-up step, done once per device);
- * make that first call before any stream capture.
+ * array's device address (a host-side set-up step, done once per device and
+ * CUDA context: after a device reset the next call looks it up again in the
+ * new context); make that first call before any stream capture.  A CUDA
+ * error that an earlier, unrelated call left pending makes this call return
+ * HTTM_ERR_CUDA without enqueuing anything and without clearing that error.
  *
  * Inputs (device): dev [h, N] fp32, each query's deviation from its merged
  * token (finite, >= 0 where eligible); eligible [h, N] u8, nonzero for

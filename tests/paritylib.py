@@ -151,20 +151,52 @@ def sample_out_error(res: O.OracleResult, out_g: np.ndarray, cfg: O.OracleConfig
     return max(errs), np.sqrt(nums / dens)
 
 
-def sample_slot_error(res: O.OracleResult, out_g, cfg: O.OracleConfig, slots_per_head: int, seed: int = 0):
+def shared_slot_tokens(o_slot: np.ndarray, g_slot: np.ndarray) -> np.ndarray:
+    """[h, N] bool: the tokens whose final query slot holds the same members
+    on both sides (the oracle's slot map and the GPU's exported one).  A slot
+    is identified by its members, not its number: (count, sum and minimum of
+    the member indices) of the token's slot must agree.  A near-tie that the
+    plan comparison excused moves a few tokens between slots (and renumbers
+    later singletons or outlier ranks); only the tokens of those slots drop
+    out, the output of every other token must match the oracle's."""
+    h, N = o_slot.shape
+    n = np.arange(N, dtype=np.int64)
+    ok = np.zeros((h, N), dtype=bool)
+
+    def sig(s):
+        ns = int(s.max()) + 1
+        cnt = np.bincount(s, minlength=ns)
+        tot = np.bincount(s, weights=n.astype(np.float64), minlength=ns)   # exact below 2^53
+        order = np.lexsort((n, s))
+        first = np.full(ns, N, dtype=np.int64)
+        ss = s[order]
+        start = np.r_[True, ss[1:] != ss[:-1]]
+        first[ss[start]] = n[order][start]
+        return cnt[s], tot[s], first[s]
+
+    for hh in range(h):
+        a, b = sig(np.asarray(o_slot[hh], dtype=np.int64)), sig(np.asarray(g_slot[hh], dtype=np.int64))
+        ok[hh] = (a[0] == b[0]) & (a[1] == b[1]) & (a[2] == b[2])
+    return ok
+
+
+def sample_slot_error(res: O.OracleResult, out_g, cfg: O.OracleConfig, slots_per_head: int, seed: int = 0,
+                      token_ok: np.ndarray | None = None):
     """Oracle attention for a seeded sample of the live query slots of each
     head (all of them if the head has fewer), compared at every token whose
     output comes from a sampled slot, so the unmerge's fan-out is checked as
     well.  out_g: the GPU output, a torch tensor (any device) or an array,
-    [h, N, d].  Returns (max abs error, relative L2 error, slots compared)."""
+    [h, N, d].  token_ok ([h, N] bool, optional) restricts the comparison to
+    those tokens (and the sample to slots holding one).  Returns (max abs
+    error, relative L2 error, slots compared)."""
     rng = np.random.default_rng(seed)
     h = res.restore.slot_final.shape[0]
     errs, nums, dens, n_slots = [], 0.0, 0.0, 0
     for hh in range(h):
         sf = res.restore.slot_final[hh]
-        live = np.unique(sf)                  # drained slots are read by no token
+        live = np.unique(sf if token_ok is None else sf[token_ok[hh]])   # drained slots are read by no token
         chosen = live if live.size <= slots_per_head else np.sort(rng.choice(live, slots_per_head, replace=False))
-        toks = np.nonzero(np.isin(sf, chosen))[0]
+        toks = np.nonzero(np.isin(sf, chosen) & (True if token_ok is None else token_ok[hh]))[0]
         inv = np.searchsorted(chosen, sf[toks])
         o = O.attention(res.restore.q_tilde[hh][chosen], res.k_means[hh], res.v_means[hh], cfg.softmax_scale)[inv]
         if isinstance(out_g, torch.Tensor):
@@ -178,8 +210,12 @@ def sample_slot_error(res: O.OracleResult, out_g, cfg: O.OracleConfig, slots_per
     return max(errs), np.sqrt(nums / dens), n_slots
 
 
-def run(plan: B.Plan, Q, K, V, injected=None, debug=True):
+def run(plan: B.Plan, Q, K, V, injected=None, debug=True, fields=None):
+    """One forward through the C ABI; `fields` limits the debug exports to
+    those names (the others stay NULL), all of them by default."""
     dbg = B.debug_buffers(plan) if debug else None
+    if dbg is not None and fields is not None:
+        dbg = {k: v for k, v in dbg.items() if k in fields}
     ws = plan.new_workspace()
     if injected is not None:
         out = B.httm_forward_with_plan(plan, Q, K, V, injected, dbg, workspace=ws)

@@ -141,3 +141,30 @@ def test_binding_rejects_bad_tensors_before_any_device_call():
         B.httm_forward(plan, Q.to(torch.bfloat16), Q, Q)
     with pytest.raises(ValueError, match="contiguous"):
         B.httm_forward(plan, Q.transpose(1, 2).contiguous().transpose(1, 2), Q, Q)
+
+
+def test_noalloc_binding_rejects_bad_buffers_before_the_call():
+    """httm_select_outliers_noalloc writes h * N mask bytes and h int32
+    counts and reads dev / eligible as dense [h, N] arrays: a buffer of the
+    wrong dtype, shape, layout or device is refused in Python, before any
+    pointer reaches the library."""
+    import torch
+    h, N = 3, 40
+    dev = torch.zeros((h, N), dtype=torch.float32)
+    elig = torch.zeros((h, N), dtype=torch.uint8)
+    with pytest.raises(ValueError, match="mask"):
+        B.httm_select_outliers_noalloc(dev, elig, 10, mask=torch.zeros((h, N - 1), dtype=torch.uint8))
+    with pytest.raises(ValueError, match="mask"):
+        B.httm_select_outliers_noalloc(dev, elig, 10, mask=torch.zeros((h, N), dtype=torch.int32))
+    with pytest.raises(ValueError, match="n_out"):
+        B.httm_select_outliers_noalloc(dev, elig, 10, n_out=torch.zeros((h,), dtype=torch.int64))
+    with pytest.raises(ValueError, match="n_out"):
+        B.httm_select_outliers_noalloc(dev, elig, 10, n_out=torch.zeros((h + 1,), dtype=torch.int32))
+    with pytest.raises(ValueError, match="dev must be contiguous"):
+        B.httm_select_outliers_noalloc(torch.zeros((N, h), dtype=torch.float32).t(), elig, 10)
+    with pytest.raises(ValueError, match="eligible must be contiguous"):
+        B.httm_select_outliers_noalloc(dev, torch.zeros((N, h), dtype=torch.uint8).t(), 10)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        B.httm_select_outliers_noalloc(dev, elig, 10)
+    with pytest.raises(ValueError, match="float32"):
+        B.httm_select_outliers_noalloc(dev.reshape(-1), elig, 10)

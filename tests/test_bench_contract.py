@@ -36,6 +36,8 @@ def test_reference_arm_prints_one_json_line():
     assert d["n_gpus"] == 1 and d["steps"] == 2 and d["warmup"] == 1
     assert d["value"] > 0 and d["ms_per_step"] > 0
     assert d["config"]["workload"] == "vggt_100f" and d["config"]["tokens"] == 136_900
+    from token_merging_view_b200.workloads import WORKLOADS
+    assert d["config"] == bench.workload_config(WORKLOADS["vggt_100f"], 1)   # the dict our arm prints
     assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]

@@ -38,3 +38,34 @@ def test_slot_sampling_sees_a_planted_error_in_a_fanned_out_token():
     bad[1, tok, 0] += 0.5
     mx, _, _ = PL.sample_slot_error(res, bad, cfg, 1 << 30)
     assert abs(mx - 0.5) < 1e-9
+
+
+def test_shared_slot_tokens_drops_exactly_the_moved_groups():
+    """A plan that moves one token from one group to another and renumbers
+    the slots: only the members of the two changed groups drop out, and a
+    slot renumbering alone (same members) keeps every token."""
+    cfg, res, out = _oracle()
+    o = res.restore.slot_final
+    perm = np.random.default_rng(0).permutation(int(o.max()) + 1)
+    g = perm[o]                                     # renumbered, same members
+    assert PL.shared_slot_tokens(o, g).all()
+    sf = o[2]
+    slots, counts = np.unique(sf, return_counts=True)
+    a, b = slots[np.argsort(-counts)[:2]]           # two merged groups
+    mover = np.nonzero(sf == a)[0][-1]
+    g2 = g.copy()
+    g2[2, mover] = perm[b]
+    ok = PL.shared_slot_tokens(o, g2)
+    assert ok[:2].all()
+    changed = (sf == a) | (sf == b)
+    assert np.array_equal(ok[2], ~changed)
+    # the restricted output check still sees a planted error on a kept token
+    bad = out.copy()
+    keep = np.nonzero(~changed)[0][0]
+    bad[2, keep, 1] -= 0.25
+    mx, _, _ = PL.sample_slot_error(res, bad, cfg, 1 << 30, token_ok=ok)
+    assert abs(mx - 0.25) < 1e-9
+    bad2 = out.copy()
+    bad2[2, mover, 1] -= 0.25                       # an excluded token is not compared
+    mx, _, _ = PL.sample_slot_error(res, bad2, cfg, 1 << 30, token_ok=ok)
+    assert mx < 1e-12

@@ -353,11 +353,27 @@ def httm_select_outliers_noalloc(dev, eligible, outlier_pct: int, mask=None, n_o
     (its scratch is a fixed array in the library).  dev: [h, N] fp32 CUDA
     tensor, eligible: [h, N] uint8.  Returns (mask [h, N] uint8, n_out [h]
     int32).  Calls that overlap on the GPU race (they share the scratch)."""
+    if dev.dim() != 2:
+        raise ValueError("dev must be float32 [h, N]")
     h, N = dev.shape
     if dev.dtype != torch.float32 or eligible.dtype != torch.uint8 or eligible.shape != dev.shape:
         raise ValueError("dev must be float32 [h, N] and eligible uint8 [h, N]")
     mask = torch.empty((h, N), dtype=torch.uint8, device=dev.device) if mask is None else mask
     n_out = torch.empty((h,), dtype=torch.int32, device=dev.device) if n_out is None else n_out
+    # the kernels read and write these as dense arrays of exactly these sizes
+    # on dev's device: anything else would be read in the wrong order or
+    # written out of bounds
+    if mask.dtype != torch.uint8 or tuple(mask.shape) != (h, N):
+        raise ValueError("mask must be uint8 [h, N]")
+    if n_out.dtype != torch.int32 or tuple(n_out.shape) != (h,):
+        raise ValueError("n_out must be int32 [h]")
+    bufs = (("dev", dev), ("eligible", eligible), ("mask", mask), ("n_out", n_out))
+    for name, t in bufs:
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    for name, t in bufs:
+        if not t.is_cuda or t.device != dev.device:
+            raise ValueError(f"{name} must be a CUDA tensor on {dev.device}")
     _check(load_library().httm_select_outliers_noalloc(_ptr(dev), _ptr(eligible), h, N, outlier_pct, _ptr(mask),
                                                        _ptr(n_out), _stream(stream)),
            "httm_select_outliers_noalloc")

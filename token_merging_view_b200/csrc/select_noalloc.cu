@@ -39,28 +39,6 @@ __device__ __forceinline__ uint32_t na_key(const float* dev, const uint8_t* elig
   return elig[i] ? __float_as_uint(dev[i]) + 1u : 0u;
 }
 
-// One full warp: bin of the k-th largest key and k minus the keys above it.
-__device__ void na_select_bin(const uint32_t* hist, int nb, uint32_t k, int* bin, uint32_t* krem) {
-  const int lane = threadIdx.x & 31;
-  uint32_t above = 0;
-  for (int top = nb - 1; top >= 0; top -= 32) {
-    const int bb = top - lane;
-    const uint32_t c = bb >= 0 ? hist[bb] : 0u;
-    const uint32_t inc = warp_incl_scan(c);
-    const uint32_t tot = __shfl_sync(0xffffffffu, inc, 31);
-    if (above + tot >= k) {
-      const unsigned ballot = __ballot_sync(0xffffffffu, above + inc >= k);
-      const int l = __ffs(ballot) - 1;
-      *bin = top - l;
-      *krem = k - (above + __shfl_sync(0xffffffffu, inc, l) - __shfl_sync(0xffffffffu, c, l));
-      return;
-    }
-    above += tot;
-  }
-  *bin = 0;
-  *krem = 0;
-}
-
 struct NaSel {
   int b[3];
   uint32_t k[3];
@@ -68,9 +46,9 @@ struct NaSel {
 
 __device__ void na_digits(const NaScratch* s, int passes, NaSel* out) {
   if ((threadIdx.x >> 5) != 0) return;
-  na_select_bin(s->hist[0], kHistBins, s->k, &out->b[0], &out->k[0]);
-  if (passes >= 2) na_select_bin(s->hist[1], kHistBins, out->k[0], &out->b[1], &out->k[1]);
-  if (passes >= 3) na_select_bin(s->hist[2], 1024, out->k[1], &out->b[2], &out->k[2]);
+  warp_select_bin(s->hist[0], kHistBins, s->k, &out->b[0], &out->k[0]);
+  if (passes >= 2) warp_select_bin(s->hist[1], kHistBins, out->k[0], &out->b[1], &out->k[1]);
+  if (passes >= 3) warp_select_bin(s->hist[2], 1024, out->k[1], &out->b[2], &out->k[2]);
 }
 
 __global__ void na_zero_kernel(NaScratch* s) {
@@ -233,20 +211,53 @@ __global__ void __launch_bounds__(1024) na_emit_kernel(const float* dev, const u
 }
 
 std::mutex g_setup_mu;
-std::vector<void*> g_scratch_ptr;   // device address of g_select_scratch, per device
+// Per device: the device address of g_select_scratch and the context it was
+// taken in.  A device reset (cudaDeviceReset) destroys the primary context
+// and reloads the module in the next one, which may place the array
+// elsewhere, so the address is looked up again whenever the device's current
+// context is not the one it was taken in.
+struct ScratchAddr {
+  void* ptr = nullptr;
+  void* ctx = nullptr;
+};
+std::vector<ScratchAddr> g_scratch;
 
-// Once per device, with that device current: the array's device address.
+typedef int (*CtxGetCurrentFn)(void**);   // cuCtxGetCurrent (CUresult is an int enum)
+
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
+
+// With the device current: the array's device address in the current
+// context (looked up once per device and context).  If no context is current
+// yet, the lookup itself initialises the device's primary context.
 httm_status scratch_address(NaScratch** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return HTTM_ERR_CUDA;
+  CtxGetCurrentFn get = ctx_get_current();
+  if (!get) return HTTM_ERR_CUDA;
+  void* ctx = nullptr;
+  if (get(&ctx) != 0) return HTTM_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_setup_mu);
-  if ((int)g_scratch_ptr.size() <= dev) g_scratch_ptr.resize(dev + 1, nullptr);
-  if (!g_scratch_ptr[dev]) {
+  if ((int)g_scratch.size() <= dev) g_scratch.resize(dev + 1);
+  ScratchAddr& a = g_scratch[dev];
+  if (!a.ptr || ctx == nullptr || a.ctx != ctx) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_select_scratch) != cudaSuccess || p == nullptr) return HTTM_ERR_CUDA;
-    g_scratch_ptr[dev] = p;
+    if (get(&ctx) != 0 || ctx == nullptr) return HTTM_ERR_CUDA;
+    a.ptr = p;
+    a.ctx = ctx;
   }
-  *out = static_cast<NaScratch*>(g_scratch_ptr[dev]);
+  *out = static_cast<NaScratch*>(a.ptr);
   return HTTM_OK;
 }
 
@@ -262,6 +273,9 @@ extern "C" httm_status httm_select_outliers_noalloc(const float* dev, const uint
   if (h < 1 || N < 1 || outlier_pct < 0 || outlier_pct > 100) return HTTM_ERR_ARG;
   if ((reinterpret_cast<uintptr_t>(dev) & 3u) || (reinterpret_cast<uintptr_t>(n_out) & 3u)) return HTTM_ERR_ALIGN;
   if (h > kNaMaxHeads || (long long)h * N > kNaMaxTokens) return HTTM_ERR_UNSUPPORTED;
+  // an error another call left pending is not this call's: leave it for its
+  // owner to read, and enqueue nothing
+  if (cudaPeekAtLastError() != cudaSuccess) return HTTM_ERR_CUDA;
   NaScratch* s = nullptr;
   httm_status st = scratch_address(&s);
   if (st != HTTM_OK) return st;
