@@ -2,10 +2,14 @@
 
 One step = one httm_forward over one VGGT-shaped layer: match, merge, the
 outlier filter, attention and unmerge, with Q/K/V already resident in HBM.
-value = tokens of all ranks / step time (max over ranks); each rank runs its
-own independent layer (weak scaling, no data-path collective).
+On one GPU, value = the layer's tokens / step time.  Under torchrun with N > 1
+ranks the layer is split by heads (16 / N heads per GPU, the outlier
+filter's counts summed over NCCL between its steps): value = the layer's
+tokens / step time, max over ranks (strong scaling).  --replicas instead
+runs an independent layer per GPU (value = tokens of all ranks / step time,
+weak scaling, no data-path collective).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload vggt_100f]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload vggt_100f] [--replicas]
     python bench.py --impl reference ...   # the fp64 CPU oracle on a bounded sample
     python bench.py --sweep                # 1000-frame sweep of merge / outlier ratios and plan variants
     python bench.py --block-sweep          # block shapes n_s x n_t on the 100-frame layer
@@ -45,6 +49,11 @@ def parse():
     ap.add_argument("--sweep-rows", type=int, default=128, help="sampled query rows per head for the output error")
     ap.add_argument("--block-sweep", action="store_true",
                     help="100-frame layer: spatial (n_t = 1) against spatio-temporal block shapes at three block sizes")
+    ap.add_argument("--shard-heads", action="store_true",
+                    help="run the head-sharded layer even on one rank (through httm_forward_sharded)")
+    ap.add_argument("--replicas", action="store_true",
+                    help="with N > 1 ranks: an independent layer per GPU (weak scaling) instead of one layer "
+                         "split by heads over the ranks")
     return ap.parse_args()
 
 
@@ -256,6 +265,24 @@ def measure_layer(w, steps: int, warmup: int, rank: int, world: int, dev, with_e
     plan.profile(False)
     res = {"plan": plan, "Q": Q, "K": K, "V": V, "ms_step": total_ms / steps, "stages": stages, "sum_lq": sum_lq,
            "launches": launches, "clocks": clk}
+    if with_e2e:
+        # the unmerge folded into the attention epilogue (httm_set_fused_unmerge),
+        # timed the same two ways, then switched back off
+        B.httm_set_fused_unmerge(plan, True)
+        step()
+        torch.cuda.synchronize()
+        assert B.httm_get_device_status(plan, ws) == 0
+        fused_ms = timed(step, steps) / steps
+        plan.profile(True)
+        plan.profile_read()
+        timed(step, steps)
+        fstages = plan.profile_read()
+        plan.profile(False)
+        B.httm_set_fused_unmerge(plan, False)
+        res["fused_unmerge"] = {"ms_per_step": round(fused_ms, 4), "launches": plan.launches(),
+                                "attention_ms_with_unmerge": round(fstages["attention"][0] / steps, 4),
+                                "default_attention_plus_unmerge_ms": round(
+                                    (stages["attention"][0] + stages["unmerge"][0]) / steps, 4)}
     if with_e2e:
         # Cached merge indices (LiteVGGT note, key design 3): the following
         # layers reuse the member lists the last full call left in `ws`.
@@ -485,6 +512,7 @@ def run_ours(args):
     e2e = {"value": round(world * w.N / (r["e2e_ms"] / 1e3), 1), "unit": "tokens/s",
            "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]}
     launches, clk, stages = r["launches"], r["clocks"], r["stages"]
+    fused_unmerge = r.get("fused_unmerge")
     ru = r["reuse"]
     group = ms_step + 5 * ru["ms"]          # indices computed on one layer of six, reused on five
     cached = {"ms_per_reused_layer": round(ru["ms"], 4), "launches_per_reused_layer": ru["launches"],
@@ -532,6 +560,7 @@ def run_ours(args):
                              "value and ms_per_step from the pass without (key branch beside query branch)",
             "dense_attention_same_length": dense,
             "cached_merge_indices": cached,
+            "fused_unmerge": fused_unmerge,
             "secondary_workload": secondary,
             "clocks": clk,
             "cpu_baseline": cpu,
@@ -779,14 +808,148 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------------------
+# one layer split by heads over the ranks (HTTM note, key design 3: every step
+# is per head except the outlier filter's global top-d%, whose counts the
+# ranks sum over NCCL between the filter's steps)
+# ----------------------------------------------------------------------------
+
+def shard_heads(H: int, world: int) -> int:
+    """Heads per rank of an H-head layer split over `world` ranks."""
+    if world < 1 or H % world != 0:
+        raise ValueError(f"{H} heads do not split evenly over {world} ranks")
+    return H // world
+
+
+def sharded_line(w, world: int, steps: int, warmup: int, ms_step: float, e2e_ms: float, h2d: int, d2h: int,
+                 launches: int, exchanges: int, roof: dict, stages: dict, clocks) -> dict:
+    """The bench line of a head-sharded layer: `value` counts the layer's
+    tokens once (the ranks split one layer: strong scaling)."""
+    h = shard_heads(w.h, world)
+    cfg = workload_config(w, world)
+    cfg["parallelism"] = (f"head-sharded x{world} ({h} of {w.h} heads per GPU; the outlier filter's counts "
+                          f"summed over the ranks by NCCL all-reduce)")
+    return {
+        "metric": METRIC, "value": round(w.N / (ms_step / 1e3), 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": steps, "warmup": warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None, "dtype": "f32" if w.fp32 else "bf16",
+        "data": "synthetic (seeded blurred-field Q/K/V, VGGT global-attention shapes)",
+        "config": cfg,
+        "e2e": {"value": round(w.N / (e2e_ms / 1e3), 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches, "collectives_per_step": exchanges,
+        "roofline": roof, "stage_ms_per_step_rank0": stages, "clocks": clocks,
+    }
+
+
+def run_sharded(args):
+    import torch
+    import torch.distributed as dist
+
+    from token_merging_view_b200 import binding as B
+    from token_merging_view_b200.inputs import make_qkv
+    from token_merging_view_b200.workloads import WORKLOADS
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+    w = WORKLOADS[args.workload]
+    h = shard_heads(w.h, world)
+    # every rank draws the whole layer from the same seed and keeps its heads
+    Qa, Ka, Va = make_qkv(T=w.T, grid=w.grid, h=w.h, d=w.d, seed=w.seed, noise_sigma=w.noise_sigma,
+                          max_shift=w.max_shift, dtype=torch.float32 if w.fp32 else torch.bfloat16, device=dev)
+    Q, K, V = (t[rank * h:(rank + 1) * h].contiguous() for t in (Qa, Ka, Va))
+    del Qa, Ka, Va
+    torch.cuda.empty_cache()
+    plan = B.httm_plan(B.LayerConfig.from_workload(w, h=h)).shard(rank, world)
+    ws = plan.new_workspace(dev)
+    out = torch.empty_like(Q)
+    stream = torch.cuda.current_stream()
+    ex = B.TorchExchange() if world > 1 else None
+
+    def step(q=Q, k=K, v=V, o=out, wsp=ws):
+        B.httm_forward_sharded(plan, q, k, v, ex, out=o, workspace=wsp, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert B.httm_get_device_status(plan, ws) == 0
+    n_out = B.workspace_view(plan, ws, "n_out").cpu()
+    sum_lq = h * plan.info.q_slots + int(n_out.sum())
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def timed(fn, n):
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n):
+            fn()
+        b.record(stream)
+        barrier()
+        return max_over_ranks(a.elapsed_time(b), world, dev)
+
+    calls0 = ex.calls if ex else 0
+    clocks = Clocks(dev.index if dev.index is not None else 0)
+    total_ms = timed(step, args.steps)
+    clk = clocks.stop()
+    exchanges = ((ex.calls - calls0) // args.steps) if ex else 0
+    launches = plan.launches() * args.steps * world
+    plan.profile(True)
+    plan.profile_read()
+    timed(step, args.steps)
+    stages = plan.profile_read()
+    plan.profile(False)
+    # end to end: this rank's heads of Q, K, V from pinned host memory, its
+    # output back, every step
+    hQ, hK, hV = (t.cpu().pin_memory() for t in (Q, K, V))
+    hO = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+
+    def e2e_step():
+        for t, hsrc in zip((Q, K, V), (hQ, hK, hV)):
+            t.copy_(hsrc, non_blocking=True)
+        step()
+        hO.copy_(out, non_blocking=True)
+
+    e2e_step()
+    e2e_ms = timed(e2e_step, args.steps) / args.steps
+    h2d = 3 * Q.numel() * Q.element_size() * world
+    d2h = out.numel() * out.element_size() * world
+    ms_step = total_ms / args.steps
+    att_ms, att_n = stages["attention"]
+    flops = 4.0 * w.d * plan.info.kv_slots * sum_lq
+    pk, pk_kind = peaks()
+    achieved = flops / (att_ms / max(1, att_n) / 1e3) / 1e12
+    roof = {"bound": "tensor", "kernel": "attention (attn_tc_kernel), rank 0's heads", "achieved": round(achieved, 2),
+            "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": round(achieved / pk["bf16_tflops"], 4),
+            "peak_kind": f"{pk_kind} bf16 burst", "traffic": None}
+    if rank == 0:
+        line = sharded_line(w, world, args.steps, args.warmup, ms_step, e2e_ms, h2d, d2h, launches, exchanges, roof,
+                            {k: round(v[0] / args.steps, 4) for k, v in stages.items()}, clk)
+        print(json.dumps(line), flush=True)
+    del plan, ws
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def main():
     args = parse()
+    _, world, _ = dist_env()
     if args.impl == "reference":
         run_reference(args)
     elif args.sweep:
         run_sweep(args)
     elif args.block_sweep:
         run_block_sweep(args)
+    elif (world > 1 and not args.replicas) or args.shard_heads:
+        run_sharded(args)
     else:
         run_ours(args)
 

@@ -300,6 +300,21 @@ httm_status httm_reorder(httm_plan_t plan, const void* X, void* Xb, int inverse,
 httm_status httm_set_wait_budget(httm_plan_t plan, uint64_t nanoseconds);
 
 /*
+ * httm_set_fused_unmerge: with enable != 0, later forward calls on `plan`
+ * that run the tensor-core attention (bf16, d_head = 64, merged modes) write
+ * each attention output row straight to the tokens it stands for -- the
+ * non-outlier members of its slot, or the outlier itself -- from the
+ * attention epilogue, and launch no separate unmerge kernel (HTTM note, key
+ * designs 1-2: unmerge copies a merged token's output back to its members
+ * in the original order).  The output is bit-identical to the default path;
+ * the O~ rows in the workspace are then not written.  Default 0: the
+ * attention writes O~ and an unmerge kernel copies it out (measured faster
+ * on B200: the scattered row writes lengthen every attention wave's tail).
+ * Host only; HTTM_ERR_ARG for a null plan.
+ */
+httm_status httm_set_fused_unmerge(httm_plan_t plan, int enable);
+
+/*
  * Synchronises `stream`, then reads the device status word of `workspace`
  * into *status (0 = clean; HTTM_DEV_* bits otherwise) and clears it.
  * Returns HTTM_ERR_DEVICE_BOUNDS / HTTM_ERR_TIMEOUT when bits were set.
@@ -369,6 +384,15 @@ httm_status httm_select_outliers_noalloc(const float* dev, const uint8_t* eligib
                                          int32_t outlier_pct, uint8_t* mask, int32_t* n_out, void* stream);
 
 const char* httm_status_str(httm_status s);
+
+/*
+ * After a call returned HTTM_ERR_CUDA: which launch or runtime call of the
+ * library failed and the CUDA error it met ("<call>: <error name> (<error
+ * string>)"), for the calling host thread; "" if none has failed on this
+ * thread.  The string stays valid until the thread's next call of this
+ * function.
+ */
+const char* httm_last_cuda_error(void);
 
 #ifdef __cplusplus
 }

@@ -54,3 +54,24 @@ def test_cuda_arm_fails_without_a_gpu():
     r = _bench("--steps", "1", "--warmup", "1", "--no-cpu-baseline")
     assert r.returncode != 0
     assert not any(ln.startswith("{") for ln in r.stdout.splitlines())
+
+
+def test_head_sharded_line_names_the_split():
+    """With N > 1 ranks bench.py splits one layer by heads: its line counts
+    the layer's tokens once (strong scaling) and names the split."""
+    import bench
+    from token_merging_view_b200.workloads import WORKLOADS
+    w = WORKLOADS["vggt_100f"]
+    assert [bench.shard_heads(16, n) for n in (1, 2, 4, 8, 16)] == [16, 8, 4, 2, 1]
+    for bad in (3, 5, 32):
+        with pytest.raises(ValueError):
+            bench.shard_heads(16, bad)
+    d = bench.sharded_line(w, 4, 10, 3, 5.0, 6.0, 111, 222, 100, 5, {"bound": "tensor"}, {}, None)
+    assert d["scaling"] == "strong" and d["n_gpus"] == 4 and d["higher_is_better"] is True
+    assert d["metric"] == bench.METRIC and d["unit"] == "tokens/s"
+    assert d["value"] == round(w.N / 0.005, 1) and d["ms_per_step"] == 5.0
+    assert d["e2e"] == {"value": round(w.N / 0.006, 1), "unit": "tokens/s", "h2d_bytes_per_step": 111,
+                        "d2h_bytes_per_step": 222}
+    assert d["config"]["workload"] == "vggt_100f"
+    assert d["config"]["parallelism"].startswith("head-sharded x4 (4 of 16 heads per GPU")
+    assert d["collectives_per_step"] == 5

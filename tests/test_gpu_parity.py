@@ -328,3 +328,22 @@ def test_forward_records_into_a_cuda_graph(w):
     assert torch.equal(out_g, eager2)
     assert not torch.equal(eager2, eager)
     del g
+
+
+@pytest.mark.parametrize("w", [MID, MID.with_(T=1, n_t=1), MID.with_(out_pct=100),
+                               MID.with_(mode=CONTIGUOUS, contig_block=384), WORKLOADS["vggt_30f"]],
+                         ids=["mid", "split_parts", "all_outliers", "contiguous", "vggt_30f"])
+def test_fused_unmerge_is_bit_identical(w):
+    """httm_set_fused_unmerge: the attention epilogue (and the merge of the
+    last wave's split items) writes each output row straight to its tokens
+    -- a slot's non-outlier members, or the outlier itself -- instead of O~
+    plus an unmerge kernel.  Same bits as the default path, clean status,
+    also when every eligible query is an outlier (drained slots)."""
+    _, plan, _, (Q, K, V), _ = _case(w)
+    ref = B.httm_forward(plan, Q, K, V, workspace=plan.new_workspace())
+    B.httm_set_fused_unmerge(plan, True)
+    ws = plan.new_workspace()
+    got = B.httm_forward(plan, Q, K, V, out=torch.full_like(Q, float("nan")), workspace=ws)
+    assert B.httm_get_device_status(plan, ws) == 0
+    assert torch.equal(got, ref)
+    B.httm_set_fused_unmerge(plan, False)

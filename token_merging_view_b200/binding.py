@@ -27,7 +27,7 @@ EXPORTS = (
     "httm_forward", "httm_forward_debug", "httm_forward_with_plan", "httm_forward_reuse", "httm_reorder",
     "httm_get_device_status", "httm_forward_launches", "httm_profile_enable", "httm_profile_read",
     "httm_select_outliers_noalloc", "httm_set_wait_budget", "httm_status_str",
-    "httm_plan_shard", "httm_forward_sharded",
+    "httm_plan_shard", "httm_forward_sharded", "httm_last_cuda_error", "httm_set_fused_unmerge",
 )
 STAGES = ("match", "merge", "outlier", "attention", "unmerge", "other")
 
@@ -103,11 +103,15 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.httm_select_outliers_noalloc.restype = ctypes.c_int
     lib.httm_set_wait_budget.argtypes = [P, ctypes.c_uint64]
     lib.httm_set_wait_budget.restype = ctypes.c_int
+    lib.httm_set_fused_unmerge.argtypes = [P, I]
+    lib.httm_set_fused_unmerge.restype = ctypes.c_int
     lib.httm_plan_shard.argtypes = [P, ctypes.c_int32, ctypes.c_int32]
     lib.httm_forward_sharded.argtypes = [P, V, V, V, V, V, S, ctypes.POINTER(httm_exchange),
                                          ctypes.POINTER(httm_debug), V]
     lib.httm_status_str.argtypes = [I]
     lib.httm_status_str.restype = ctypes.c_char_p
+    lib.httm_last_cuda_error.argtypes = []
+    lib.httm_last_cuda_error.restype = ctypes.c_char_p
     for name in ("httm_plan", "httm_get_plan_info", "httm_forward", "httm_forward_debug",
                  "httm_forward_with_plan", "httm_forward_reuse", "httm_reorder", "httm_get_device_status",
                  "httm_profile_enable", "httm_profile_read", "httm_plan_shard", "httm_forward_sharded"):
@@ -118,7 +122,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
 
 class HttmError(RuntimeError):
     def __init__(self, status: int, where: str):
-        msg = load_library().httm_status_str(status).decode()
+        lib = load_library()
+        msg = lib.httm_status_str(status).decode()
+        if status == 6:                                   # HTTM_ERR_CUDA: which call, which error
+            detail = lib.httm_last_cuda_error().decode()
+            if detail:
+                msg += f" [{detail}]"
         super().__init__(f"{where}: {msg} (status {status})")
         self.status = status
 
@@ -319,6 +328,12 @@ def httm_set_wait_budget(plan: Plan, nanoseconds: int) -> None:
     (default 2e9 ns); 0 makes every wait that is not already complete run
     out (HTTM_DEV_TIMEOUT), for checking the failure path."""
     _check(load_library().httm_set_wait_budget(plan.handle, int(nanoseconds)), "httm_set_wait_budget")
+
+
+def httm_set_fused_unmerge(plan: Plan, enable: bool) -> None:
+    """Write attention output rows straight to their tokens from the
+    attention epilogue (no separate unmerge launch) on later calls."""
+    _check(load_library().httm_set_fused_unmerge(plan.handle, int(bool(enable))), "httm_set_fused_unmerge")
 
 
 def httm_get_device_status(plan: Plan, workspace, stream=None) -> int:

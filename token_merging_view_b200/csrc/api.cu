@@ -4,6 +4,7 @@
 #include <algorithm>
 #include <atomic>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <new>
 #include <vector>
@@ -36,6 +37,7 @@ struct httm_plan_s {
   std::vector<int4> items_h;
   // stage timing
   bool profile = false;
+  bool fused_unmerge = false;   // httm_set_fused_unmerge
   struct Rec { int stage; int n; cudaEvent_t a, b; };
   std::vector<Rec> recs;
   std::vector<cudaEvent_t> pool;
@@ -80,11 +82,40 @@ cudaError_t launch_attention_simt(const Dims& dims, bool fp32, const void* q, co
                                   void* o, int Lk, const Buffers& buf, cudaStream_t s);
 bool attention_tc_supported(const Dims& dims, bool fp32);
 cudaError_t launch_attention_tc(const Dims& dims, const void* q, const void* k, const void* v, void* o,
-                                int Lk, const Buffers& buf, cudaStream_t s);
+                                int Lk, const Buffers& buf, cudaStream_t s, void* unmerge_out);
 bool match_tc_supported(const Dims& dims, bool fp32);
 }  // namespace httm
 
 namespace {
+
+// The last CUDA error a call of this library met on this thread, for
+// httm_last_cuda_error().
+thread_local cudaError_t t_last_err = cudaSuccess;
+thread_local const char* t_last_where = "";
+
+httm_status cuda_fail(cudaError_t e, const char* where) {
+  t_last_err = e;
+  t_last_where = where;
+  return HTTM_ERR_CUDA;
+}
+
+// HTTM_SYNC_CHECK=1 in the environment: synchronise the stream after every
+// launch, so that a fault is attributed to the kernel that raised it (a
+// debugging aid; it serialises the forward).
+bool sync_check() {
+  static const bool on = [] {
+    const char* v = getenv("HTTM_SYNC_CHECK");
+    return v && v[0] == '1';
+  }();
+  return on;
+}
+
+cudaError_t checked(cudaError_t e, cudaStream_t s) {
+  if (e != cudaSuccess || !sync_check()) return e;
+  (void)s;
+  const cudaError_t e2 = cudaDeviceSynchronize();    // every stream of the call (the key branch too)
+  return e2 != cudaSuccess ? e2 : cudaGetLastError();
+}
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -226,50 +257,61 @@ httm_status check_device(httm_plan_s* plan) {
 
 #define HTTM_LAUNCH(expr)                             \
   do {                                                \
-    cudaError_t e_ = (expr);                          \
+    cudaError_t e_ = checked((expr), s);              \
     ++launches;                                       \
-    if (e_ != cudaSuccess) return HTTM_ERR_CUDA;      \
+    if (e_ != cudaSuccess) return cuda_fail(e_, #expr); \
   } while (0)
 
 // The attention stage: the tensor-core kernel plus the merge of the last
 // wave's split items (two launches, timed as one stage), or the CUDA-core
-// kernel.  Adds its launches to *launches.
+// kernel.  With `unmerge_out` (a merged layer on the tensor-core path) the
+// tensor-core kernels write every output row straight to the tokens it
+// stands for in unmerge_out and *fused is set: no unmerge launch follows.
+// Adds its launches to *launches.
 httm_status attention(const httm_plan_s* plan, const void* q, const void* k, const void* v, void* o, int Lk,
-                      const Buffers& buf, cudaStream_t s, int* launches) {
+                      const Buffers& buf, cudaStream_t s, int* launches, void* unmerge_out = nullptr,
+                      bool* fused = nullptr) {
   cudaError_t e;
+  if (fused) *fused = false;
   if (attention_tc_supported(plan->dims, plan->fp32)) {
-    e = launch_attention_tc(plan->dims, q, k, v, o, Lk, buf, s);
+    e = launch_attention_tc(plan->dims, q, k, v, o, Lk, buf, s, unmerge_out);
     *launches += 2;
+    if (fused) *fused = unmerge_out != nullptr;
   } else {
     e = launch_attention_simt(plan->dims, plan->fp32, q, k, v, o, Lk, buf, s);
     *launches += 1;
   }
-  return e == cudaSuccess ? HTTM_OK : HTTM_ERR_CUDA;
+  e = checked(e, s);
+  return e == cudaSuccess ? HTTM_OK : cuda_fail(e, "attention");
 }
 
-// The outlier filter (without its restore).  With a collective (a
-// head-sharded layer), the shards sum the eligible count and the first
-// histogram (both built by the query gather), each later histogram, and the
-// per-shard counts of keys equal to the threshold, between the steps.
-httm_status outlier_stage(const Dims& dims, bool fp32, const void* Q, bool mask_inj, const Buffers& buf,
-                          cudaStream_t s, const httm_exchange* ex, int* launches) {
+// The outlier filter and its restore.  With a collective (a head-sharded
+// layer), the shards sum the eligible count and the first histogram (both
+// built by the query gather), each later histogram, and the per-shard counts
+// of keys equal to the threshold, between the steps.
+httm_status filter_stage(const httm_plan_s* plan, const void* Q, bool mask_inj, const Buffers& buf, const Debug& dd,
+                         cudaStream_t s, const httm_exchange* ex, int* launches) {
+  const Dims& dims = plan->dims;
+  const bool fp32 = plan->fp32;
   if (!ex) {
-    const cudaError_t e = launch_outlier(dims, fp32, Q, mask_inj, buf, s);
+    if (cudaError_t e_ = checked(launch_outlier(dims, fp32, Q, mask_inj, buf, s), s); e_ != cudaSuccess) return cuda_fail(e_, "launch_outlier");
     *launches += mask_inj ? 3 : 5;  // two histogram passes, count, scan, emit
-    return e == cudaSuccess ? HTTM_OK : HTTM_ERR_CUDA;
-  }
-  auto sum = [&](void* p, int64_t n, int32_t eb) { return ex->allreduce_sum(p, n, eb, s, ex->user) == 0; };
-  if (!sum(&buf.state->n_eligible, 1, 4) || !sum(buf.hist, kHistBins, 4)) return HTTM_ERR_EXCHANGE;
-  for (int pass = 2; pass <= 3; ++pass) {
-    if (launch_outlier_pass(dims, buf, pass, s) != cudaSuccess) return HTTM_ERR_CUDA;
+  } else {
+    auto sum = [&](void* p, int64_t n, int32_t eb) { return ex->allreduce_sum(p, n, eb, s, ex->user) == 0; };
+    if (!sum(&buf.state->n_eligible, 1, 4) || !sum(buf.hist, kHistBins, 4)) return HTTM_ERR_EXCHANGE;
+    for (int pass = 2; pass <= 3; ++pass) {
+      if (cudaError_t e_ = checked(launch_outlier_pass(dims, buf, pass, s), s); e_ != cudaSuccess) return cuda_fail(e_, "launch_outlier_pass");
+      ++*launches;
+      if (!sum(buf.hist + (pass - 1) * kHistBins, pass == 2 ? kHistBins : 1024, 4)) return HTTM_ERR_EXCHANGE;
+    }
+    if (cudaError_t e_ = checked(launch_outlier_count(dims, false, buf, s), s); e_ != cudaSuccess) return cuda_fail(e_, "launch_outlier_count");
     ++*launches;
-    if (!sum(buf.hist + (pass - 1) * kHistBins, pass == 2 ? kHistBins : 1024, 4)) return HTTM_ERR_EXCHANGE;
+    if (!sum(buf.hist + 3 * kHistBins, kMaxShards, 4)) return HTTM_ERR_EXCHANGE;
+    if (cudaError_t e_ = checked(launch_outlier_emit(dims, fp32, Q, false, buf, s), s); e_ != cudaSuccess) return cuda_fail(e_, "launch_outlier_emit");
+    *launches += 2;  // scan, emit
   }
-  if (launch_outlier_count(dims, false, buf, s) != cudaSuccess) return HTTM_ERR_CUDA;
+  if (cudaError_t e_ = checked(launch_restore(dims, fp32, plan->blocks_d, Q, buf, dd, s), s); e_ != cudaSuccess) return cuda_fail(e_, "launch_restore");
   ++*launches;
-  if (!sum(buf.hist + 3 * kHistBins, kMaxShards, 4)) return HTTM_ERR_EXCHANGE;
-  if (launch_outlier_emit(dims, fp32, Q, false, buf, s) != cudaSuccess) return HTTM_ERR_CUDA;
-  *launches += 2;  // scan, emit
   return HTTM_OK;
 }
 
@@ -340,13 +382,14 @@ httm_status forward_impl(httm_plan_s* plan, const void* Q, const void* K, const 
     HTTM_LAUNCH(launch_merge(dims, fp32, plan->blocks_d, plan_inj, reuse, Q, K, V, buf, dd, s, 1));
     HTTM_LAUNCH(launch_merge(dims, fp32, plan->blocks_d, plan_inj, reuse, Q, K, V, buf, dd, s2, 2));
     if (!reuse) launches += 2;  // the two planning launches
-    if ((st = outlier_stage(dims, fp32, Q, mask_inj, buf, s, ex, &launches)) != HTTM_OK) return st;
-    HTTM_LAUNCH(launch_restore(dims, fp32, plan->blocks_d, Q, buf, dd, s));
+    if ((st = filter_stage(plan, Q, mask_inj, buf, dd, s, ex, &launches)) != HTTM_OK) return st;
     if (cudaEventRecord(plan->ev_join, s2) != cudaSuccess || cudaStreamWaitEvent(s, plan->ev_join, 0) != cudaSuccess)
       return HTTM_ERR_CUDA;
-    st = attention(plan, buf.q_tilde, buf.k_tilde, buf.v_tilde, buf.o_tilde, dims.k_slots, buf, s, &launches);
+    bool fused = false;
+    st = attention(plan, buf.q_tilde, buf.k_tilde, buf.v_tilde, buf.o_tilde, dims.k_slots, buf, s, &launches,
+                   plan->fused_unmerge ? out : nullptr, &fused);
     if (st != HTTM_OK) return st;
-    HTTM_LAUNCH(launch_unmerge(dims, fp32, buf, out, s));
+    if (!fused) HTTM_LAUNCH(launch_unmerge(dims, fp32, buf, out, s));
     if (dbg) HTTM_LAUNCH(launch_export(dims, plan->blocks_d, buf, dd, s));
     plan->launches = launches;
     return HTTM_OK;
@@ -359,7 +402,8 @@ httm_status forward_impl(httm_plan_s* plan, const void* Q, const void* K, const 
     else
       e = launch_match_simt(dims, fp32, plan->blocks_d, plan->match_items_d, plan->n_match_items, Q, K, buf, s);
     ++launches;
-    if (e != cudaSuccess) return HTTM_ERR_CUDA;
+    e = checked(e, s);
+    if (e != cudaSuccess) return cuda_fail(e, "matching");
   }
   {
     StageTimer t(plan, s, HTTM_STAGE_MERGE, reuse ? 2 : 3);
@@ -367,16 +411,21 @@ httm_status forward_impl(httm_plan_s* plan, const void* Q, const void* K, const 
     launches += reuse ? 1 : 2;  // planning (unless reused), then the two gathers
   }
   {
-    StageTimer t(plan, s, HTTM_STAGE_OUTLIER, mask_inj ? 4 : 6);
-    if ((st = outlier_stage(dims, fp32, Q, mask_inj, buf, s, ex, &launches)) != HTTM_OK) return st;
-    HTTM_LAUNCH(launch_restore(dims, fp32, plan->blocks_d, Q, buf, dd, s));
+    const int before = launches;
+    StageTimer t(plan, s, HTTM_STAGE_OUTLIER, 0);
+    if ((st = filter_stage(plan, Q, mask_inj, buf, dd, s, ex, &launches)) != HTTM_OK) return st;
+    t.n = launches - before;
   }
+  bool fused = false;
   {
+    // with the unmerge fused into the attention epilogue, its time (and its
+    // writes of the output) fall in this stage
     StageTimer t(plan, s, HTTM_STAGE_ATTENTION, 1);
-    st = attention(plan, buf.q_tilde, buf.k_tilde, buf.v_tilde, buf.o_tilde, dims.k_slots, buf, s, &launches);
+    st = attention(plan, buf.q_tilde, buf.k_tilde, buf.v_tilde, buf.o_tilde, dims.k_slots, buf, s, &launches,
+                   plan->fused_unmerge ? out : nullptr, &fused);
     if (st != HTTM_OK) return st;
   }
-  {
+  if (!fused) {
     StageTimer t(plan, s, HTTM_STAGE_UNMERGE, 1);
     HTTM_LAUNCH(launch_unmerge(dims, fp32, buf, out, s));
   }
@@ -671,9 +720,22 @@ httm_status httm_get_device_status(httm_plan_t plan, void* workspace, void* stre
 
 int32_t httm_forward_launches(httm_plan_t plan) { return plan ? plan->launches : -1; }
 
+const char* httm_last_cuda_error(void) {
+  static thread_local char msg[256];
+  if (t_last_err == cudaSuccess) return "";
+  snprintf(msg, sizeof(msg), "%s: %s (%s)", t_last_where, cudaGetErrorName(t_last_err), cudaGetErrorString(t_last_err));
+  return msg;
+}
+
 httm_status httm_set_wait_budget(httm_plan_t plan, uint64_t nanoseconds) {
   if (!plan) return HTTM_ERR_ARG;
   plan->dims.wait_budget_ns = nanoseconds;
+  return HTTM_OK;
+}
+
+httm_status httm_set_fused_unmerge(httm_plan_t plan, int enable) {
+  if (!plan) return HTTM_ERR_ARG;
+  plan->fused_unmerge = enable != 0;
   return HTTM_OK;
 }
 

@@ -60,17 +60,68 @@ constexpr int kThreads = 384;
 constexpr uint32_t kTile = kBN * kD * 2;   // 16 KB: 128 rows x 64 bf16
 constexpr uint32_t kColO = 384;             // O_t at kColO + 64 t; S ring buffers at 0, 128, 256
 
+constexpr int kListCap = 8;                 // output tokens of a query row kept in shared memory
+
 struct AttnSmem {
   uint8_t q[2][kTile];
   uint8_t k[kStages][kTile];
   uint8_t v[kStages][kTile];
+  int lst_tok[kAttnRows][kListCap];         // fused unmerge: the tokens each query row's output goes to
+  int lst_n[kAttnRows];                     // ... how many (more than kListCap: walk the member list)
   uint64_t q_full;
   uint64_t kv_full[kStages], kv_empty[kStages];
   uint64_t s_full[3], p_full[2], o_done[2];
+  uint64_t lists_full;
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
 };
+
+// Fused unmerge: where the rows of O~ go.  out == null: the kernel writes
+// the O~ rows and a separate unmerge kernel copies them out.  Otherwise
+// every output row is written straight to the tokens it stands for in
+// out [h, N, 64] -- the non-outlier members of a regular slot, or the
+// outlier itself (HTTM note, key designs 1-2: unmerge copies a merged
+// token's output back to each member, in the original order) -- and O~ is
+// not written.
+struct Scatter {
+  __nv_bfloat16* out;
+  int N;
+  long long out_base;                       // first outlier row of Q~
+};
+
+// The tokens whose output is row gr of O~ (head hh), in member order;
+// calls put(tok) for each.  Members that are outliers take their own row.
+template <class F>
+__device__ __forceinline__ void row_targets(const Buffers& buf, const Scatter& sc, int hh, long long gr, F&& put) {
+  const size_t tb = (size_t)hh * sc.N;
+  if (gr >= sc.out_base) {
+    const int tok = buf.o_tok[gr - sc.out_base];
+    if (tok >= 0 && tok < sc.N) put(tok);
+    else set_status(buf.state, HTTM_DEV_BOUNDS);
+    return;
+  }
+  const int c = buf.q_gcount[gr], gs = buf.q_gstart[gr];
+  if (c < 0 || gs < 0 || gs + c > sc.N) {
+    set_status(buf.state, HTTM_DEV_BOUNDS);
+    return;
+  }
+  for (int j = 0; j < c; ++j) {
+    const int tok = buf.q_members[tb + gs + j];
+    if (tok < 0 || tok >= sc.N) {
+      set_status(buf.state, HTTM_DEV_BOUNDS);
+      continue;
+    }
+    if (buf.mask[tb + tok] == 0) put(tok);
+  }
+}
+
+__device__ __forceinline__ void put_row(const Scatter& sc, int hh, int tok, const uint32_t (&packed)[32]) {
+  uint4* dst = reinterpret_cast<uint4*>(sc.out + ((size_t)hh * sc.N + tok) * kD);
+#pragma unroll
+  for (int v = 0; v < 8; ++v)
+    dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+}
 constexpr size_t kSmemBytes = sizeof(AttnSmem) + 1024;
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 
@@ -101,7 +152,7 @@ __device__ __forceinline__ SplitPlan split_plan(int n, int S, int n_kv) {
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                const __grid_constant__ CUtensorMap tv, __nv_bfloat16* __restrict__ O, int Lk, float scale_log2,
-               int n_sm, Buffers buf) {
+               int n_sm, Buffers buf, Scatter sc) {
   const int n_kv_all = (Lk + kBN - 1) / kBN;
   const SplitPlan sp = split_plan((int)buf.state->n_items, n_sm, n_kv_all);
   const int n_cta = sp.n_full + sp.r * sp.p;
@@ -137,6 +188,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
       mbar_init(&sm.o_done[t], 1);
     }
     mbar_init(&sm.drain, 1);
+    mbar_init(&sm.lists_full, 64);
     sm.abort = 0;
     mbar_fence_init();
   }
@@ -215,6 +267,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
       // every MMA issued above completes before TMEM is released
       umma_commit(&sm.drain);
       drain_wait(&sm.drain, 0);
+    } else if ((warp == 2 || warp == 3) && sc.out != nullptr && part < 0) {
+      // ---------------------------------------------------- unmerge targets
+      // while the main loop runs: each query row's output tokens into
+      // shared memory (the epilogue then writes without a global lookup)
+      for (int r = threadIdx.x - 64; r < kAttnRows; r += 64) {
+        int n = 0;
+        if (r < n_rows)
+          row_targets(buf, sc, hh, (long long)q_row0 + r, [&](int tok) {
+            if (n < kListCap) sm.lst_tok[r][n] = tok;
+            ++n;
+          });
+        sm.lst_n[r] = n;
+      }
+      mbar_arrive(&sm.lists_full);
     }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 208;" ::: "memory");
@@ -365,7 +431,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
           packed[c * 16 + i] = pack_bf16(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
       }
       const int r = t * kBM + row;
-      if (r < n_rows) {
+      if (sc.out != nullptr) {
+        // fused unmerge: the row goes to each token it stands for
+        if (__all_sync(0xffffffffu, mbar_wait(&sm.lists_full, 0, abort, st)) && r < n_rows) {
+          const int n = sm.lst_n[r];
+          if (n <= kListCap) {
+            for (int j = 0; j < n; ++j) put_row(sc, hh, sm.lst_tok[r][j], packed);
+          } else {
+            row_targets(buf, sc, hh, (long long)q_row0 + r, [&](int tok) { put_row(sc, hh, tok, packed); });
+          }
+        }
+      } else if (r < n_rows) {
         uint4* dst = reinterpret_cast<uint4*>(O + ((size_t)q_row0 + r) * kD);
 #pragma unroll
         for (int v = 0; v < 8; ++v)
@@ -390,7 +466,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
 // max in use, O = sum_p O_p 2^(m_p - M) / sum_p l_p 2^(m_p - M), in part
 // order; rows past the item's end are left alone.
 __global__ void __launch_bounds__(kAttnRows)
-attn_combine_kernel(__nv_bfloat16* __restrict__ O, int Lk, int n_sm, Buffers buf) {
+attn_combine_kernel(__nv_bfloat16* __restrict__ O, int Lk, int n_sm, Buffers buf, Scatter sc) {
   if (plan_failed(buf.state)) return;
   const SplitPlan sp = split_plan((int)buf.state->n_items, n_sm, (Lk + kBN - 1) / kBN);
   for (int i = blockIdx.x; i < sp.r; i += gridDim.x) {
@@ -407,7 +483,7 @@ attn_combine_kernel(__nv_bfloat16* __restrict__ O, int Lk, int n_sm, Buffers buf
         l = fmaf(src[q][kD], w[q], l);
       }
       const float inv = 1.f / l;
-      uint4* dst = reinterpret_cast<uint4*>(O + ((size_t)it.y + r) * kD);
+      uint32_t packed[32];
 #pragma unroll
       for (int v = 0; v < 8; ++v) {
         float a[8];
@@ -421,8 +497,18 @@ attn_combine_kernel(__nv_bfloat16* __restrict__ O, int Lk, int n_sm, Buffers buf
           a[4] = fmaf(x1.x, w[q], a[4]); a[5] = fmaf(x1.y, w[q], a[5]);
           a[6] = fmaf(x1.z, w[q], a[6]); a[7] = fmaf(x1.w, w[q], a[7]);
         }
-        dst[v] = make_uint4(pack_bf16(a[0] * inv, a[1] * inv), pack_bf16(a[2] * inv, a[3] * inv),
-                            pack_bf16(a[4] * inv, a[5] * inv), pack_bf16(a[6] * inv, a[7] * inv));
+        packed[4 * v] = pack_bf16(a[0] * inv, a[1] * inv);
+        packed[4 * v + 1] = pack_bf16(a[2] * inv, a[3] * inv);
+        packed[4 * v + 2] = pack_bf16(a[4] * inv, a[5] * inv);
+        packed[4 * v + 3] = pack_bf16(a[6] * inv, a[7] * inv);
+      }
+      if (sc.out != nullptr) {
+        row_targets(buf, sc, it.x, (long long)it.y + r, [&](int tok) { put_row(sc, it.x, tok, packed); });
+      } else {
+        uint4* dst = reinterpret_cast<uint4*>(O + ((size_t)it.y + r) * kD);
+#pragma unroll
+        for (int v = 0; v < 8; ++v)
+          dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
       }
     }
   }
@@ -468,7 +554,7 @@ bool attention_tc_supported(const Dims& dims, bool fp32) {
 }
 
 cudaError_t launch_attention_tc(const Dims& dims, const void* q, const void* k, const void* v, void* o, int Lk,
-                                const Buffers& buf, cudaStream_t s) {
+                                const Buffers& buf, cudaStream_t s, void* unmerge_out) {
   CUtensorMap tq, tk, tv;
   const uint64_t q_rows = dims.mode == HTTM_DENSE ? (uint64_t)dims.h * dims.N : (uint64_t)dims.q_rows_alloc;
   const uint64_t kv_rows = (uint64_t)dims.h * Lk;
@@ -485,11 +571,12 @@ cudaError_t launch_attention_tc(const Dims& dims, const void* q, const void* k, 
     return cudaErrorInvalidValue;
   const int S = std::min(n_sm, kMaxAttnParts);
   // up to S extra CTAs for the split parts of the last wave
+  const Scatter sc{static_cast<__nv_bfloat16*>(unmerge_out), dims.N, dims.out_base};
   attn_tc_kernel<<<dims.max_items + S, kThreads, kSmemBytes, s>>>(tq, tk, tv, static_cast<__nv_bfloat16*>(o), Lk,
-                                                                  scale_log2, S, buf);
+                                                                  scale_log2, S, buf, sc);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  attn_combine_kernel<<<S, kAttnRows, 0, s>>>(static_cast<__nv_bfloat16*>(o), Lk, S, buf);
+  attn_combine_kernel<<<S, kAttnRows, 0, s>>>(static_cast<__nv_bfloat16*>(o), Lk, S, buf, sc);
   return cudaGetLastError();
 }
 

@@ -50,12 +50,12 @@ __device__ void block_select(const uint32_t* hist, int nb, uint32_t k, uint32_t*
     *krem = 0;
   }
   uint32_t s = 0;
-  for (int i = 0; i < per; ++i) s += hist[top - i];
+  for (int i = 0; i < per; ++i) s += __ldcg(hist + top - i);   // built by other CTAs: read at L2
   uint32_t tot;
   uint32_t above = block_excl_scan(s, tmp, &tot);
   if (above < k && k <= above + s) {
     for (int i = 0; i < per; ++i) {
-      const uint32_t c = hist[top - i];
+      const uint32_t c = __ldcg(hist + top - i);
       if (k <= above + c) {
         *bin = top - i;
         *krem = k - above;
