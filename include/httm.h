@@ -24,7 +24,8 @@
  *    access instead of trapping.  Each forward call clears the word when it
  *    starts; httm_get_device_status() reads it.
  *  - Nothing throws across this boundary.  The library allocates no device
- *    memory except the small block table owned by a plan.
+ *    memory except the small block table owned by a plan (and, for an
+ *    HTTM_PARTITION plan, its token classes and block lists).
  *  - A plan is not thread-safe: calls on one plan from several host threads
  *    must not overlap (the caller serialises them, or gives each thread a
  *    plan of its own; plans are cheap).  Calls on different plans may run
@@ -60,6 +61,7 @@ typedef enum {
   HTTM_HEAD_UNIFORM = 1,      /* one plan per block from the head-mean cosine, used by all heads */
   HTTM_CONTIGUOUS = 2,        /* per-head plans inside runs of contig_block tokens, no reorder */
   HTTM_DENSE = 3,             /* no merging: plain softmax attention over all N tokens */
+  HTTM_PARTITION = 4,         /* HTTM blocks with LiteVGGT's destination rule (httm_plan_partition) */
 } httm_mode;
 
 /* Device status word bits (httm_get_device_status). */
@@ -75,6 +77,7 @@ typedef enum {
  *                    per head; d_head in {16, 64}.  The tensor-core kernels
  *                    serve bf16 with d_head = 64; other shapes run on
  *                    CUDA-core kernels (a correctness path for small cases).
+ *                    HTTM_PARTITION needs bf16 with d_head = 64.
  *  n_s, n_t          block = n_s consecutive patches (raster) x n_t frames;
  *                    the last region / temporal group may be partial.
  *  contig_block      block length of HTTM_CONTIGUOUS (ignored otherwise).
@@ -277,6 +280,42 @@ httm_status httm_plan_shard(httm_plan_t plan, int32_t shard, int32_t shards);
 httm_status httm_forward_sharded(httm_plan_t plan, const void* Q, const void* K, const void* V, void* out,
                                  void* workspace, size_t workspace_bytes, const httm_exchange* ex,
                                  const httm_debug* dbg, void* stream);
+
+/*
+ * httm_plan_partition: LiteVGGT's token partition as the destination rule
+ * of an HTTM_PARTITION plan ("LiteVGGT: Boosting Vanilla VGGT via
+ * Geometry-aware Cached Token Merging", key designs 1-2).  `score` is a
+ * DEVICE array [T, P] fp32, one geometric-importance score per token
+ * (shared by the heads; the note derives it from image gradients and local
+ * variance -- here the caller supplies it).  Per frame the
+ * floor(ga_pct * P / 100) highest scores are geometry-aware (GA) tokens that
+ * never merge (score ties: lower patch index first); the first frame's
+ * other tokens are all destinations; in every later frame the lowest-
+ * scoring non-GA token of each 2x2 cell of the grid x grid patch grid (P =
+ * grid^2; cells from even rows and columns, 2x1 / 1x2 / 1x1 on an odd edge;
+ * ties: lower patch index) is a destination; the other tokens are sources.
+ * Merging stays per head inside the plan's temporal blocks (n_s x n_t): a
+ * block's destinations are the destination-class tokens in it, every source
+ * merges into its most similar one (cosine, ties to the lowest destination
+ * in block order), GA tokens (and the sources of a block without
+ * destinations) stay single.  Q and K use the same classes; V follows K.
+ * The plan's q/kv strides and merge ratios are ignored in this mode.
+ * The classes and per-block lists are computed on the device; the call then
+ * SYNCHRONISES `stream` to read the per-block counts (2 ints a block) and
+ * resizes the plan: call httm_get_plan_info / httm_workspace_bytes again
+ * afterwards.  It may be called again with a new score (the plan then
+ * holds the new partition).  roles_out (optional DEVICE [T, P] u8) receives
+ * the classes: 0 source, 1 destination, 2 GA.  The first call binds the plan
+ * to the current device and allocates its class / list arrays (N bytes +
+ * 8 N bytes, owned by the plan).  Errors: HTTM_ERR_ARG (not an
+ * HTTM_PARTITION plan, null score, ga_pct outside [0, 100], P not a square);
+ * HTTM_ERR_UNSUPPORTED (P > 16384, or a block with more than 1280
+ * destinations).  Forward calls on an HTTM_PARTITION plan return
+ * HTTM_ERR_ARG until it has been partitioned; httm_forward_with_plan and
+ * httm_plan_shard do not support this mode (HTTM_ERR_UNSUPPORTED).
+ */
+httm_status httm_plan_partition(httm_plan_t plan, const float* score, int32_t ga_pct, uint8_t* roles_out,
+                                void* stream);
 
 /*
  * httm_reorder: temporal reordering (key design 2).  inverse = 0: X in

@@ -168,3 +168,27 @@ def test_noalloc_binding_rejects_bad_buffers_before_the_call():
         B.httm_select_outliers_noalloc(dev, elig, 10)
     with pytest.raises(ValueError, match="float32"):
         B.httm_select_outliers_noalloc(dev.reshape(-1), elig, 10)
+
+
+def test_partition_plan_host_checks():
+    """HTTM_PARTITION: bf16 with d_head = 64 only; a plan that has not been
+    partitioned refuses forward calls and sharding; the partition call
+    refuses other modes (host checks, no device call)."""
+    import ctypes
+    w = WORKLOADS["tiny_4f_8x8"]
+    with pytest.raises(B.HttmError) as e:
+        B.httm_plan(B.LayerConfig.from_workload(w, mode=B.HTTM_PARTITION))      # fp32, d_head 16
+    assert e.value.status == 2
+    cfg = B.LayerConfig(h=2, T=3, P=64, d_head=64, mode=B.HTTM_PARTITION, n_s=16, n_t=2,
+                        q_dst_stride=0, kv_dst_stride=0, q_merge_pct=-1, kv_merge_pct=-1)   # ignored in this mode
+    plan = B.httm_plan(cfg)
+    lib = B.load_library()
+    fake = ctypes.c_void_p(1 << 20)
+    assert lib.httm_forward(plan.handle, fake, fake, fake, fake, fake, 1 << 40, None) == 1
+    assert lib.httm_plan_shard(plan.handle, 0, 2) == 2
+    other = B.httm_plan(B.LayerConfig.from_workload(WORKLOADS["vggt_30f"]))
+    assert lib.httm_plan_partition(other.handle, fake, 10, None, None) == 1
+    assert lib.httm_plan_partition(plan.handle, None, 10, None, None) == 1
+    assert lib.httm_plan_partition(plan.handle, fake, 101, None, None) == 1
+    bad = B.httm_plan(B.LayerConfig(h=2, T=3, P=60, d_head=64, mode=B.HTTM_PARTITION, n_s=16, n_t=2))
+    assert lib.httm_plan_partition(bad.handle, fake, 10, None, None) == 1       # 60 patches: not a square grid

@@ -18,7 +18,7 @@ from .workloads import Workload
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libhttm.so")
 
 HTTM_BF16, HTTM_F32 = 0, 1
-HTTM_HEADWISE_TEMPORAL, HTTM_HEAD_UNIFORM, HTTM_CONTIGUOUS, HTTM_DENSE = 0, 1, 2, 3
+HTTM_HEADWISE_TEMPORAL, HTTM_HEAD_UNIFORM, HTTM_CONTIGUOUS, HTTM_DENSE, HTTM_PARTITION = 0, 1, 2, 3, 4
 HTTM_DEV_BAD_PLAN, HTTM_DEV_BOUNDS, HTTM_DEV_TIMEOUT = 0x1, 0x2, 0x4
 
 # every symbol include/httm.h declares
@@ -28,6 +28,7 @@ EXPORTS = (
     "httm_get_device_status", "httm_forward_launches", "httm_profile_enable", "httm_profile_read",
     "httm_select_outliers_noalloc", "httm_set_wait_budget", "httm_status_str",
     "httm_plan_shard", "httm_forward_sharded", "httm_last_cuda_error", "httm_set_fused_unmerge",
+    "httm_plan_partition",
 )
 STAGES = ("match", "merge", "outlier", "attention", "unmerge", "other")
 
@@ -105,6 +106,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.httm_set_wait_budget.restype = ctypes.c_int
     lib.httm_set_fused_unmerge.argtypes = [P, I]
     lib.httm_set_fused_unmerge.restype = ctypes.c_int
+    lib.httm_plan_partition.argtypes = [P, V, ctypes.c_int32, V, V]
+    lib.httm_plan_partition.restype = ctypes.c_int
     lib.httm_plan_shard.argtypes = [P, ctypes.c_int32, ctypes.c_int32]
     lib.httm_forward_sharded.argtypes = [P, V, V, V, V, V, S, ctypes.POINTER(httm_exchange),
                                          ctypes.POINTER(httm_debug), V]
@@ -328,6 +331,28 @@ def httm_set_wait_budget(plan: Plan, nanoseconds: int) -> None:
     (default 2e9 ns); 0 makes every wait that is not already complete run
     out (HTTM_DEV_TIMEOUT), for checking the failure path."""
     _check(load_library().httm_set_wait_budget(plan.handle, int(nanoseconds)), "httm_set_wait_budget")
+
+
+def httm_plan_partition(plan: Plan, score, ga_pct: int = 10, roles_out=None, stream=None):
+    """LiteVGGT's token partition as the destination rule of an
+    HTTM_PARTITION plan: ``score`` is a [T, P] float32 CUDA tensor (one
+    geometric-importance score per token).  Synchronises the stream and
+    resizes the plan (its workspace size changes).  Returns the token
+    classes [T, P] uint8 (0 source, 1 destination, 2 GA)."""
+    T, P = plan.cfg.T, plan.cfg.P
+    if score.dtype != torch.float32 or tuple(score.shape) != (T, P) or not score.is_contiguous():
+        raise ValueError(f"score must be a contiguous float32 [{T}, {P}] tensor")
+    if roles_out is None:
+        roles_out = torch.empty((T, P), dtype=torch.uint8, device=score.device)
+    if roles_out.dtype != torch.uint8 or tuple(roles_out.shape) != (T, P) or not roles_out.is_contiguous():
+        raise ValueError(f"roles_out must be a contiguous uint8 [{T}, {P}] tensor")
+    lib = load_library()
+    _check(lib.httm_plan_partition(plan.handle, _ptr(score), int(ga_pct), _ptr(roles_out), _stream(stream)),
+           "httm_plan_partition")
+    info = httm_plan_info()
+    _check(lib.httm_get_plan_info(plan.handle, ctypes.byref(info)), "httm_get_plan_info")
+    plan.info = info
+    return roles_out
 
 
 def httm_set_fused_unmerge(plan: Plan, enable: bool) -> None:

@@ -38,6 +38,12 @@ struct httm_plan_s {
   // stage timing
   bool profile = false;
   bool fused_unmerge = false;   // httm_set_fused_unmerge
+  // HTTM_PARTITION: token classes, block lists, list ordinals, per-block counts
+  bool partitioned = false;
+  uint8_t* roles_d = nullptr;
+  int32_t* lists_d = nullptr;
+  int32_t* ord_d = nullptr;
+  int32_t* counts_d = nullptr;
   struct Rec { int stage; int n; cudaEvent_t a, b; };
   std::vector<Rec> recs;
   std::vector<cudaEvent_t> pool;
@@ -324,6 +330,8 @@ httm_status forward_impl(httm_plan_s* plan, const void* Q, const void* K, const 
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(out)) return HTTM_ERR_ALIGN;
   if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return HTTM_ERR_ALIGN;
   if (reuse && (inj || plan->dims.mode == HTTM_DENSE)) return HTTM_ERR_ARG;
+  if (plan->dims.mode == HTTM_PARTITION && !plan->partitioned) return HTTM_ERR_ARG;
+  if (plan->dims.mode == HTTM_PARTITION && inj) return HTTM_ERR_UNSUPPORTED;
   if (ws_bytes < plan->ws.total) return HTTM_ERR_WORKSPACE;
   if (inj) {
     const bool any = inj->q_best || inj->q_merged || inj->k_best || inj->k_merged;
@@ -437,6 +445,81 @@ httm_status forward_impl(httm_plan_s* plan, const void* Q, const void* K, const 
   return HTTM_OK;
 }
 
+// From each block's destination / merge counts (q_ndst, k_ndst, q_r, k_r):
+// the source and slot offsets, the plan's sizes and outlier budget, and the
+// matching work lists (CUDA-core: 128-source tiles of every (tensor, block);
+// tensor cores: one CTA per (tensor, head, block), a block split in runs of
+// whole 128-source tiles when that gives too few CTAs; costliest first).
+void finish_blocks(httm_plan_s* p) {
+  const httm_cfg& c = p->cfg;
+  Dims& d = p->dims;
+  std::vector<BlockDesc>& B = p->blocks_h;
+  int qs = 0, ks = 0, qsl = 0, ksl = 0;
+  d.max_ndst = d.max_nsrc = d.max_nb = 0;
+  for (BlockDesc& b : B) {
+    b.q_src_off = qs;
+    b.k_src_off = ks;
+    b.q_slot_off = qsl;
+    b.k_slot_off = ksl;
+    qs += b.n_b - b.q_ndst;
+    ks += b.n_b - b.k_ndst;
+    qsl += b.n_b - b.q_r;
+    ksl += b.n_b - b.k_r;
+    d.max_ndst = std::max(d.max_ndst, std::max(b.q_ndst, b.k_ndst));
+    d.max_nsrc = std::max(d.max_nsrc, std::max(b.n_b - b.q_ndst, b.n_b - b.k_ndst));
+    d.max_nb = std::max(d.max_nb, b.n_b);
+  }
+  d.q_src = qs;
+  d.k_src = ks;
+  d.q_slots = qsl;
+  d.k_slots = ksl;
+  size_outliers(d, c.outlier_pct);
+  std::vector<int4> items;
+  for (int t = 0; t < 2; ++t)
+    for (int bi = 0; bi < d.nblk; ++bi) {
+      const BlockDesc& b = B[bi];
+      const int ns = b.n_b - (t == 0 ? b.q_ndst : b.k_ndst);
+      for (int s0 = 0; s0 < ns; s0 += 128) items.push_back(make_int4(t, bi, s0, std::min(128, ns - s0)));
+    }
+  std::stable_sort(items.begin(), items.end(), [&](const int4& a, const int4& b) {
+    const int ca = a.x == 0 ? B[a.y].q_ndst : B[a.y].k_ndst;
+    const int cb = b.x == 0 ? B[b.y].q_ndst : B[b.y].k_ndst;
+    return ca > cb;
+  });
+  p->n_match_items = (int)items.size();
+  p->items_h = std::move(items);
+  // (head-uniform: one item list for all heads, item.x = tensor; a block
+  // without destinations, possible under HTTM_PARTITION, needs no matching)
+  std::vector<int4> tci;
+  const int hs = c.mode == HTTM_HEAD_UNIFORM ? 1 : c.h;
+  const int parts_want = std::max(1, (4 * 148 + 2 * d.nblk * hs - 1) / (2 * d.nblk * hs));
+  for (int hh = 0; hh < hs; ++hh)
+    for (int t = 0; t < 2; ++t)
+      for (int bi = 0; bi < d.nblk; ++bi) {
+        const BlockDesc& b = B[bi];
+        const int nd = t == 0 ? b.q_ndst : b.k_ndst;
+        if (nd == 0) continue;
+        const int ns = b.n_b - nd;
+        const int tiles = (ns + 127) / 128;
+        const int parts = std::max(1, std::min(parts_want, tiles));
+        const int per = (tiles + parts - 1) / parts;
+        for (int t0 = 0; t0 < tiles; t0 += per) {
+          const int s0 = t0 * 128, n = std::min(per * 128, ns - s0);
+          tci.push_back(make_int4(t + 2 * hh, bi, s0, n));
+        }
+      }
+  // query items first, then key items; each costliest first
+  std::stable_sort(tci.begin(), tci.end(), [&](const int4& a, const int4& b) {
+    if ((a.x & 1) != (b.x & 1)) return (a.x & 1) < (b.x & 1);
+    const long long ca = (long long)((a.x & 1) == 0 ? B[a.y].q_ndst : B[a.y].k_ndst) * a.w;
+    const long long cb = (long long)((b.x & 1) == 0 ? B[b.y].q_ndst : B[b.y].k_ndst) * b.w;
+    return ca > cb;
+  });
+  p->n_tc_q = (int)std::count_if(tci.begin(), tci.end(), [](const int4& a) { return (a.x & 1) == 0; });
+  p->n_tc_items = (int)tci.size();
+  p->tc_items_h = std::move(tci);
+}
+
 }  // namespace
 
 extern "C" {
@@ -463,14 +546,17 @@ httm_status httm_plan(const httm_cfg* cfg, httm_plan_t* out) {
   const httm_cfg c = *cfg;
   if (c.h < 1 || c.h > 64 || c.T < 1 || c.P < 1) return HTTM_ERR_ARG;
   if (c.dtype != HTTM_BF16 && c.dtype != HTTM_F32) return HTTM_ERR_ARG;
-  if (c.mode < HTTM_HEADWISE_TEMPORAL || c.mode > HTTM_DENSE) return HTTM_ERR_ARG;
+  if (c.mode < HTTM_HEADWISE_TEMPORAL || c.mode > HTTM_PARTITION) return HTTM_ERR_ARG;
+  if (c.mode == HTTM_PARTITION && (c.dtype != HTTM_BF16 || c.d_head != 64)) return HTTM_ERR_UNSUPPORTED;
   if (c.d_head != 16 && c.d_head != 64) return HTTM_ERR_UNSUPPORTED;
   if (c.softmax_scale < 0.f) return HTTM_ERR_ARG;
   const long long N = (long long)c.T * c.P;
   if (N > (1ll << 30) || (long long)c.h * N > (1ll << 31) - 1) return HTTM_ERR_UNSUPPORTED;
   if (c.mode != HTTM_DENSE) {
-    if (c.q_dst_stride < 2 || c.kv_dst_stride < 2) return HTTM_ERR_ARG;
-    if (c.q_merge_pct < 0 || c.q_merge_pct > 100 || c.kv_merge_pct < 0 || c.kv_merge_pct > 100) return HTTM_ERR_ARG;
+    if (c.mode != HTTM_PARTITION) {          // the partition fixes destinations and merges itself
+      if (c.q_dst_stride < 2 || c.kv_dst_stride < 2) return HTTM_ERR_ARG;
+      if (c.q_merge_pct < 0 || c.q_merge_pct > 100 || c.kv_merge_pct < 0 || c.kv_merge_pct > 100) return HTTM_ERR_ARG;
+    }
     if (c.outlier_pct < 0 || c.outlier_pct > 100) return HTTM_ERR_ARG;
     if (c.mode == HTTM_CONTIGUOUS ? c.contig_block < 1 : (c.n_s < 1 || c.n_t < 1)) return HTTM_ERR_ARG;
   }
@@ -527,13 +613,15 @@ httm_status httm_plan(const httm_cfg* cfg, httm_plan_t* out) {
         }
       }
     }
-    int tok = 0, qs = 0, ks = 0, qsl = 0, ksl = 0;
+    int tok = 0;
     for (BlockDesc& b : B) {
       if (b.n_b > 8192) {
         delete p;
         return HTTM_ERR_UNSUPPORTED;
       }
       b.tok_off = tok;
+      tok += b.n_b;
+      if (c.mode == HTTM_PARTITION) continue;     // destinations come from httm_plan_partition
       b.q_ndst = (b.n_b + c.q_dst_stride - 1) / c.q_dst_stride;
       b.k_ndst = (b.n_b + c.kv_dst_stride - 1) / c.kv_dst_stride;
       b.q_r = (int)(((long long)c.q_merge_pct * b.n_b) / 100);
@@ -542,69 +630,9 @@ httm_status httm_plan(const httm_cfg* cfg, httm_plan_t* out) {
         delete p;
         return HTTM_ERR_INFEASIBLE_RATIO;
       }
-      b.q_src_off = qs;
-      b.k_src_off = ks;
-      b.q_slot_off = qsl;
-      b.k_slot_off = ksl;
-      tok += b.n_b;
-      qs += b.n_b - b.q_ndst;
-      ks += b.n_b - b.k_ndst;
-      qsl += b.n_b - b.q_r;
-      ksl += b.n_b - b.k_r;
-      d.max_ndst = std::max(d.max_ndst, std::max(b.q_ndst, b.k_ndst));
-      d.max_nsrc = std::max(d.max_nsrc, std::max(b.n_b - b.q_ndst, b.n_b - b.k_ndst));
-      d.max_nb = std::max(d.max_nb, b.n_b);
     }
     d.nblk = (int32_t)B.size();
-    d.q_src = qs;
-    d.k_src = ks;
-    d.q_slots = qsl;
-    d.k_slots = ksl;
-    size_outliers(d, c.outlier_pct);
-    // matching work: 128-source tiles of every (tensor, block), costliest first
-    std::vector<int4> items;
-    for (int t = 0; t < 2; ++t)
-      for (int bi = 0; bi < d.nblk; ++bi) {
-        const BlockDesc& b = B[bi];
-        const int ns = b.n_b - (t == 0 ? b.q_ndst : b.k_ndst);
-        for (int s0 = 0; s0 < ns; s0 += 128) items.push_back(make_int4(t, bi, s0, std::min(128, ns - s0)));
-      }
-    std::stable_sort(items.begin(), items.end(), [&](const int4& a, const int4& b) {
-      const int ca = a.x == 0 ? B[a.y].q_ndst : B[a.y].k_ndst;
-      const int cb = b.x == 0 ? B[b.y].q_ndst : B[b.y].k_ndst;
-      return ca > cb;
-    });
-    p->n_match_items = (int)items.size();
-    p->items_h = std::move(items);
-    // tensor-core matching: one CTA per (tensor, head, block), a block split in
-    // runs of whole 128-source tiles when that gives too few CTAs; costliest first
-    // (head-uniform: one item list for all heads, item.x = tensor)
-    std::vector<int4> tci;
-    const int hs = c.mode == HTTM_HEAD_UNIFORM ? 1 : c.h;
-    const int parts_want = std::max(1, (4 * 148 + 2 * d.nblk * hs - 1) / (2 * d.nblk * hs));
-    for (int hh = 0; hh < hs; ++hh)
-      for (int t = 0; t < 2; ++t)
-        for (int bi = 0; bi < d.nblk; ++bi) {
-          const BlockDesc& b = B[bi];
-          const int ns = b.n_b - (t == 0 ? b.q_ndst : b.k_ndst);
-          const int tiles = (ns + 127) / 128;
-          const int parts = std::max(1, std::min(parts_want, tiles));
-          const int per = (tiles + parts - 1) / parts;
-          for (int t0 = 0; t0 < tiles; t0 += per) {
-            const int s0 = t0 * 128, n = std::min(per * 128, ns - s0);
-            tci.push_back(make_int4(t + 2 * hh, bi, s0, n));
-          }
-        }
-    // query items first, then key items; each costliest first
-    std::stable_sort(tci.begin(), tci.end(), [&](const int4& a, const int4& b) {
-      if ((a.x & 1) != (b.x & 1)) return (a.x & 1) < (b.x & 1);
-      const long long ca = (long long)((a.x & 1) == 0 ? B[a.y].q_ndst : B[a.y].k_ndst) * a.w;
-      const long long cb = (long long)((b.x & 1) == 0 ? B[b.y].q_ndst : B[b.y].k_ndst) * b.w;
-      return ca > cb;
-    });
-    p->n_tc_q = (int)std::count_if(tci.begin(), tci.end(), [](const int4& a) { return (a.x & 1) == 0; });
-    p->n_tc_items = (int)tci.size();
-    p->tc_items_h = std::move(tci);
+    if (c.mode != HTTM_PARTITION) finish_blocks(p);
   }
   p->ws = layout(d, p->fp32);
   *out = p;
@@ -621,6 +649,10 @@ void httm_plan_destroy(httm_plan_t plan) {
   if (plan->blocks_d) cudaFree(plan->blocks_d);
   if (plan->match_items_d) cudaFree(plan->match_items_d);
   if (plan->tc_items_d) cudaFree(plan->tc_items_d);
+  if (plan->roles_d) cudaFree(plan->roles_d);
+  if (plan->lists_d) cudaFree(plan->lists_d);
+  if (plan->ord_d) cudaFree(plan->ord_d);
+  if (plan->counts_d) cudaFree(plan->counts_d);
   if (plan->side) cudaStreamDestroy(plan->side);
   if (plan->ev_fork) cudaEventDestroy(plan->ev_fork);
   if (plan->ev_join) cudaEventDestroy(plan->ev_join);
@@ -675,6 +707,7 @@ httm_status httm_plan_shard(httm_plan_t plan, int32_t shard, int32_t shards) {
   if (!plan || shards < 1 || shards > kMaxShards || shard < 0 || shard >= shards || plan->device >= 0)
     return HTTM_ERR_ARG;
   if (plan->dims.mode == HTTM_HEAD_UNIFORM && shards > 1) return HTTM_ERR_UNSUPPORTED;
+  if (plan->dims.mode == HTTM_PARTITION) return HTTM_ERR_UNSUPPORTED;
   Dims d = plan->dims;
   d.shard = shard;
   d.shards = shards;
@@ -691,6 +724,77 @@ httm_status httm_forward_sharded(httm_plan_t plan, const void* Q, const void* K,
                                  void* workspace, size_t workspace_bytes, const httm_exchange* ex,
                                  const httm_debug* dbg, void* stream) {
   return forward_impl(plan, Q, K, V, out, workspace, workspace_bytes, nullptr, dbg, stream, false, true, ex);
+}
+
+httm_status httm_plan_partition(httm_plan_t plan, const float* score, int32_t ga_pct, uint8_t* roles_out,
+                                void* stream) {
+  if (!plan || !score || plan->dims.mode != HTTM_PARTITION || ga_pct < 0 || ga_pct > 100) return HTTM_ERR_ARG;
+  const httm_cfg& c = plan->cfg;
+  int grid = 0;
+  while ((grid + 1) * (grid + 1) <= c.P) ++grid;
+  if (grid * grid != c.P) return HTTM_ERR_ARG;
+  if (c.P > 16384) return HTTM_ERR_UNSUPPORTED;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return HTTM_ERR_CUDA;
+  if (plan->device >= 0 && plan->device != dev) return HTTM_ERR_ARG;
+  Dims& d = plan->dims;
+  const size_t N = (size_t)d.N;
+  const size_t nb = plan->blocks_h.size();
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (!plan->roles_d) {
+    if (cudaMalloc(&plan->roles_d, N) != cudaSuccess || cudaMalloc(&plan->lists_d, N * 4) != cudaSuccess ||
+        cudaMalloc(&plan->ord_d, N * 4) != cudaSuccess || cudaMalloc(&plan->counts_d, nb * 8) != cudaSuccess ||
+        (!plan->blocks_d && cudaMalloc(&plan->blocks_d, nb * sizeof(BlockDesc)) != cudaSuccess))
+      return HTTM_ERR_CUDA;
+  }
+  // the block geometry (base, s, n_b, tok_off) is all the lists kernel reads
+  if (cudaMemcpy(plan->blocks_d, plan->blocks_h.data(), nb * sizeof(BlockDesc), cudaMemcpyHostToDevice) != cudaSuccess)
+    return HTTM_ERR_CUDA;
+  const int ga_k = (int)(((long long)ga_pct * c.P) / 100);
+  if (cudaError_t e = launch_partition(d, c.T, grid, ga_k, score, plan->blocks_d, plan->roles_d, plan->lists_d,
+                                       plan->ord_d, plan->counts_d, s);
+      e != cudaSuccess)
+    return cuda_fail(e, "launch_partition");
+  if (roles_out && cudaMemcpyAsync(roles_out, plan->roles_d, N, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+    return HTTM_ERR_CUDA;
+  std::vector<int32_t> counts(2 * nb);
+  if (cudaError_t e = cudaStreamSynchronize(s); e != cudaSuccess) return cuda_fail(e, "launch_partition (sync)");
+  if (cudaMemcpy(counts.data(), plan->counts_d, nb * 8, cudaMemcpyDeviceToHost) != cudaSuccess) return HTTM_ERR_CUDA;
+  // every source merges into its best destination, if its block has one
+  for (size_t i = 0; i < nb; ++i) {
+    BlockDesc& b = plan->blocks_h[i];
+    const int n_dst = counts[2 * i], n_src = counts[2 * i + 1];
+    if (n_dst < 0 || n_src < 0 || n_dst + n_src > b.n_b) return HTTM_ERR_DEVICE_BOUNDS;
+    b.q_ndst = b.k_ndst = n_dst;
+    b.q_r = b.k_r = n_dst > 0 ? n_src : 0;
+  }
+  finish_blocks(plan);
+  if (d.max_ndst > 1280) return HTTM_ERR_UNSUPPORTED;   // the matching kernel stages <= 1280 destination rows
+  d.proles = plan->roles_d;
+  d.plists = plan->lists_d;
+  d.pord = plan->ord_d;
+  // upload the sized block table and the matching work list
+  const size_t nt = std::max<size_t>(1, plan->tc_items_h.size()) * sizeof(int4);
+  if (plan->tc_items_d) cudaFree(plan->tc_items_d);
+  plan->tc_items_d = nullptr;
+  if (cudaMemcpy(plan->blocks_d, plan->blocks_h.data(), nb * sizeof(BlockDesc), cudaMemcpyHostToDevice) != cudaSuccess ||
+      cudaMalloc(&plan->tc_items_d, nt) != cudaSuccess ||
+      (!plan->tc_items_h.empty() &&
+       cudaMemcpy(plan->tc_items_d, plan->tc_items_h.data(), plan->tc_items_h.size() * sizeof(int4),
+                  cudaMemcpyHostToDevice) != cudaSuccess))
+    return HTTM_ERR_CUDA;
+  if (plan->device < 0) {
+    if (cudaStreamCreateWithFlags(&plan->side, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&plan->ev_fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&plan->ev_join, cudaEventDisableTiming) != cudaSuccess)
+      return HTTM_ERR_CUDA;
+    // the CUDA-core matching list is not used in this mode; a one-entry buffer keeps the invariants
+    if (cudaMalloc(&plan->match_items_d, sizeof(int4)) != cudaSuccess) return HTTM_ERR_CUDA;
+    plan->device = dev;
+  }
+  plan->ws = layout(d, plan->fp32);
+  plan->partitioned = true;
+  return HTTM_OK;
 }
 
 httm_status httm_reorder(httm_plan_t plan, const void* X, void* Xb, int inverse, void* stream) {

@@ -40,7 +40,16 @@ struct Dims {
   uint32_t plan_id;              // stamps a workspace whose member lists this plan wrote
   uint64_t wait_budget_ns;       // bound of a device wait (httm_set_wait_budget; default 2 s)
   int32_t shard, shards;         // head sharding: this shard holds heads [shard h, shard h + h) of h shards
+  // HTTM_PARTITION (LiteVGGT's destination rule): per token its class and its
+  // ordinal in its block's list; per block, at its tok_off, the in-block
+  // indices of its destinations (ascending) then of the others (ascending).
+  // Null in the other modes, whose destinations are the i % stride == 0.
+  const uint8_t* proles;
+  const int32_t* plists;
+  const int32_t* pord;
 };
+
+constexpr uint8_t kRoleSrc = 0, kRoleDst = 1, kRoleGA = 2;   // token classes of HTTM_PARTITION
 
 constexpr int kChunk = 4096;       // keys per chunk of the outlier compaction
 constexpr int kHistBins = 2048;    // radix digit of the outlier select (11 bits)

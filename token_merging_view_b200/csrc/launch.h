@@ -73,6 +73,12 @@ cudaError_t launch_unmerge(const Dims& dims, bool fp32, const Buffers& buf, void
 cudaError_t launch_reorder(const Dims& dims, bool fp32, const BlockDesc* blocks, const void* X,
                            void* Xb, bool inverse, cudaStream_t s);
 
+// HTTM_PARTITION: token classes from the score [T, P] (ga_k GA tokens per
+// frame), then every block's destination / other lists, each token's
+// ordinal in its list and per block (destinations, sources) in counts.
+cudaError_t launch_partition(const Dims& dims, int T, int grid, int ga_k, const float* score, const BlockDesc* blocks,
+                             uint8_t* roles, int32_t* lists, int32_t* ord, int32_t* counts, cudaStream_t s);
+
 cudaError_t launch_export(const Dims& dims, const BlockDesc* blocks, const Buffers& buf,
                           const Debug& dbg, cudaStream_t s);
 

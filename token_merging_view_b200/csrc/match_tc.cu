@@ -36,13 +36,13 @@ using namespace tc;
 constexpr int kEpiThreads = 512;
 constexpr int kParts = kEpiThreads / 128;  // epilogue warps per TMEM lane quarter
 constexpr int kThreads = kEpiThreads + 32;
-constexpr int kMaxDst = 1024;          // destination rows a block may have on this path
+constexpr int kMaxDst = 1280;          // destination rows a block may have on this path
 constexpr int kChunkCols = 256;
 constexpr uint32_t kRowsTile = 128;
 constexpr uint32_t kTileBytes = kRowsTile * 128;
 
 struct MatchSmem {
-  uint8_t dst[kMaxDst * 128];          // K-major SW128, 128 KB
+  uint8_t dst[kMaxDst * 128];          // K-major SW128, 160 KB
   uint8_t src[2][kTileBytes];
   float inv_d[kMaxDst];
   float best_v[kParts][128];
@@ -143,10 +143,13 @@ match_tc_kernel(Dims dims, const BlockDesc* __restrict__ blocks, const int4* __r
     // ------------------------------------------------------ gather + epilogue
     const uint32_t dst_addr = smem_u32(sm.dst);
     // destinations (rows padded with zeros to a multiple of 64)
+    // in-block indices: i % stride == 0 are the destinations; under
+    // HTTM_PARTITION the block's lists name them (destinations, then the rest)
+    const int32_t* bl = dims.plists ? dims.plists + b.tok_off : nullptr;
     for (int e = tid; e < ndst_pad * 8; e += kEpiThreads) {
       const int r = e >> 3, ch = e & 7;
       const bool valid = r < ndst;
-      const int tok = valid ? block_token(b, r * stride, dims.P) : b.base;
+      const int tok = valid ? block_token(b, bl ? bl[r] : r * stride, dims.P) : b.base;
       cp_async16(dst_addr + swz(r, ch), Xh + (size_t)tok * 64 + ch * 8, valid);
     }
     auto load_tile = [&](int t) {
@@ -155,7 +158,7 @@ match_tc_kernel(Dims dims, const BlockDesc* __restrict__ blocks, const int4* __r
         const int r = e >> 3, ch = e & 7;
         const int k = src0 + t * kRowsTile + r;
         const bool valid = t * (int)kRowsTile + r < nsrc;
-        const int tok = valid ? block_token(b, src_index(k, stride), dims.P) : b.base;
+        const int tok = valid ? block_token(b, bl ? bl[ndst + k] : src_index(k, stride), dims.P) : b.base;
         cp_async16(base + swz(r, ch), Xh + (size_t)tok * 64 + ch * 8, valid);
       }
     };

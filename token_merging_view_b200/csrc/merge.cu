@@ -141,10 +141,27 @@ plan_kernel(Dims dims, const BlockDesc* __restrict__ blocks, Buffers buf, Debug 
   }
   __syncthreads();
 
+  // HTTM_PARTITION: the block's lists give the in-block index of
+  // destination a (bl[a]) and of source ordinal k (bl[ndst + k])
+  const int32_t* bl = dims.plists ? dims.plists + b.tok_off : nullptr;
+
   // 1. top-r: the r sources with the largest (score, -ordinal) merge.  The
   //    r-th largest ordered score T comes from the radix select; all keys
   //    above T merge, and of the keys equal to T the lowest ordinals.
-  if (!injected) {
+  //    HTTM_PARTITION: every source-class token merges (r of them when the
+  //    block has destinations, else none); GA tokens stay single.
+  if (bl && !injected) {
+    uint32_t cnt = 0;
+    for (int k = lo; k < hi; ++k) {
+      const bool m = r > 0 && dims.proles[block_token(b, bl[ndst + k], dims.P)] == kRoleSrc;
+      mf[k] = m ? 1 : 0;
+      merged[k] = m ? 1 : 0;
+      cnt += m;
+    }
+    uint32_t tot;
+    block_excl_scan(cnt, tmp, &tot);
+    if (tid == 0 && tot != (uint32_t)r) s_bad = 1;
+  } else if (!injected) {
     uint32_t T = 0, need = 0;
     if (r > 0) {
       uint32_t prefix = 0, krem = (uint32_t)r;
@@ -254,15 +271,15 @@ plan_kernel(Dims dims, const BlockDesc* __restrict__ blocks, Buffers buf, Debug 
     if (q < ndst + r) {
       const int a = pm[q], j = q - (gsm[a] + a);
       if (j == 0) {
-        idx = a * stride;
+        idx = bl ? bl[a] : a * stride;
       } else {
         const int k = mem[gsm[a] + j - 1], g = (int)by_gap.div(k);
-        idx = g * stride + (k - g * (stride - 1)) + 1;    // in-block index of source ordinal k
+        idx = bl ? bl[ndst + k] : g * stride + (k - g * (stride - 1)) + 1;   // in-block index of source ordinal k
       }
       slot = slot_off + a;
     } else {
       const int p = q - ndst - r, k = mem[r + p], g = (int)by_gap.div(k);
-      idx = g * stride + (k - g * (stride - 1)) + 1;
+      idx = bl ? bl[ndst + k] : g * stride + (k - g * (stride - 1)) + 1;
       slot = slot_off + ndst + p;
     }
     const int tau = (int)by_s.div(idx);
@@ -688,10 +705,17 @@ __global__ void export_kernel(Dims dims, const BlockDesc* __restrict__ blocks, B
       const int stride = tensor == 0 ? dims.q_stride : dims.kv_stride;
       int bt = -1, mg = 0;
       float sc = 0.f;
-      if (i % stride != 0) {
+      // HTTM_PARTITION: a token's class says whether it is a destination,
+      // its ordinal places it in its list; a block without destinations
+      // has no match (best -1)
+      const bool part = dims.plists != nullptr;
+      const bool is_dst = part ? dims.proles[n] == kRoleDst : i % stride == 0;
+      const int ndst = tensor == 0 ? b.q_ndst : b.k_ndst;
+      if (!is_dst && (!part || ndst > 0)) {
         const size_t si = (size_t)hh * (tensor == 0 ? dims.q_src : dims.k_src) +
-                          (tensor == 0 ? b.q_src_off : b.k_src_off) + src_ordinal(i, stride);
-        bt = block_token(b, (tensor == 0 ? buf.q_best : buf.k_best)[si] * stride, dims.P);
+                          (tensor == 0 ? b.q_src_off : b.k_src_off) + (part ? dims.pord[n] : src_ordinal(i, stride));
+        const int m = (tensor == 0 ? buf.q_best : buf.k_best)[si];
+        bt = block_token(b, part ? dims.plists[b.tok_off + m] : m * stride, dims.P);
         sc = (tensor == 0 ? buf.q_score : buf.k_score)[si];
         mg = (tensor == 0 ? buf.q_merged : buf.k_merged)[si];
       }

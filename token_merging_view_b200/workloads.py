@@ -10,7 +10,7 @@ seeded generator settings of :mod:`token_merging_view_b200.inputs`.
 
 Modes: 0 = head-wise temporal (HTTM), 1 = head-uniform (one plan per block
 from the head-mean cosine), 2 = contiguous blocks in the original order,
-3 = dense (no merging).
+3 = dense (no merging), 4 = HTTM blocks with LiteVGGT's destination rule.
 """
 from __future__ import annotations
 
@@ -20,6 +20,7 @@ HEADWISE_TEMPORAL = 0
 HEAD_UNIFORM = 1
 CONTIGUOUS = 2
 DENSE = 3
+PARTITION = 4
 
 
 @dataclass(frozen=True)
