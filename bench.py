@@ -49,6 +49,9 @@ def parse():
     ap.add_argument("--sweep-rows", type=int, default=128, help="sampled query rows per head for the output error")
     ap.add_argument("--block-sweep", action="store_true",
                     help="100-frame layer: spatial (n_t = 1) against spatio-temporal block shapes at three block sizes")
+    ap.add_argument("--skewed", action="store_true",
+                    help="100-frame layer with identical query and key tokens: every source of a block picks the "
+                         "same destination (one group of ~2,700 members per block and head)")
     ap.add_argument("--shard-heads", action="store_true",
                     help="run the head-sharded layer even on one rank (through httm_forward_sharded)")
     ap.add_argument("--replicas", action="store_true",
@@ -939,6 +942,56 @@ def run_sharded(args):
         dist.destroy_process_group()
 
 
+def run_skewed(args):
+    """The degenerate case of the merge plan: Q and K identical across every
+    token of a head (V as usual), so every cosine ties, every source takes
+    its block's first destination (lowest index) and the top-r merge puts
+    ~70 % of each block into one group.  Times the layer with stage timing
+    next to the regular layer."""
+    import torch
+
+    from token_merging_view_b200 import binding as B
+    from token_merging_view_b200.inputs import make_qkv
+    from token_merging_view_b200.workloads import WORKLOADS
+
+    rank, world, local = dist_env()
+    if rank != 0:
+        return
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = WORKLOADS[args.workload]
+    Q, K, V = make_qkv(T=w.T, grid=w.grid, h=w.h, d=w.d, seed=w.seed, noise_sigma=w.noise_sigma,
+                       max_shift=w.max_shift, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+    clocks = Clocks(dev.index if dev.index is not None else 0)
+    lines = {}
+    for name, (q, k) in (("regular", (Q, K)),
+                         ("identical_qk", (Q[:, :1].expand_as(Q).contiguous(), K[:, :1].expand_as(K).contiguous()))):
+        plan = B.httm_plan(B.LayerConfig.from_workload(w))
+        ws = plan.new_workspace(dev)
+        out = torch.empty_like(Q)
+        for _ in range(args.warmup):
+            B.httm_forward(plan, q, k, V, out=out, workspace=ws, stream=stream)
+        torch.cuda.synchronize()
+        status = B.httm_get_device_status(plan, ws)
+        steps = max(3, args.steps)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            B.httm_forward(plan, q, k, V, out=out, workspace=ws, stream=stream)
+        b.record(stream)
+        torch.cuda.synchronize()
+        plan.profile(True)
+        plan.profile_read()
+        for _ in range(steps):
+            B.httm_forward(plan, q, k, V, out=out, workspace=ws, stream=stream)
+        stages = {kk: round(v[0] / steps, 4) for kk, v in plan.profile_read().items()}
+        lines[name] = {"status": status, "ms_per_step": round(a.elapsed_time(b) / steps, 3), "stage_ms": stages}
+        del ws, plan
+        torch.cuda.empty_cache()
+    print(json.dumps({"skewed_groups": w.name, **lines, "clocks": clocks.stop()}), flush=True)
+
+
 def main():
     args = parse()
     _, world, _ = dist_env()
@@ -948,6 +1001,8 @@ def main():
         run_sweep(args)
     elif args.block_sweep:
         run_block_sweep(args)
+    elif args.skewed:
+        run_skewed(args)
     elif (world > 1 and not args.replicas) or args.shard_heads:
         run_sharded(args)
     else:

@@ -89,7 +89,8 @@ struct SmallDiv {
 // token of the block is the member of exactly one slot.  Every phase is
 // spread evenly over the threads: the top-r threshold by a 4-digit radix
 // select (8-bit digits), group sizes by shared-memory counting, each merged
-// source's place in its group by counting the group's smaller ordinals, and
+// source's place in its group by counting the group's smaller ordinals (or,
+// when a group exceeds 64 members, by ranks taken in source order), and
 // the member list written position by position (a binary search over the
 // group starts finds each position's group).
 __global__ void __launch_bounds__(kMergeThreads)
@@ -224,10 +225,44 @@ plan_kernel(Dims dims, const BlockDesc* __restrict__ blocks, Buffers buf, Debug 
     return;
   }
   block_scan_array(cm, gsm, ndst, tmp);
+  // the largest group decides how merged sources find their place: by
+  // counting the group's smaller ordinals (cheap for the usual few members),
+  // or, past 64 members (near-identical tokens put most of a block in one
+  // group), in source order, warp after warp, ranked within a warp by
+  // __match_any_sync -- the same ascending order without the c^2 cost
+  int cmax_local = 0;
+  for (int m = tid; m < ndst; m += bd) cmax_local = max(cmax_local, cm[m]);
+  cmax_local = __reduce_max_sync(0xffffffffu, cmax_local);
+  if ((tid & 31) == 0) tmp[tid >> 5] = (uint32_t)cmax_local;
+  __syncthreads();
+  int cmax_all = 0;
+  for (int w = 0; w < (bd >> 5); ++w) cmax_all = max(cmax_all, (int)tmp[w]);
+  const bool big_groups = cmax_all > 64;
   for (int m = tid; m < ndst; m += bd) cur[m] = gsm[m];
   __syncthreads();
-  for (int k = tid; k < nsrc; k += bd)
-    if (mf[k]) aux[atomicAdd(&cur[bst[k]], 1)] = k;
+  if (big_groups) {
+    const unsigned lt = (1u << (tid & 31)) - 1u;
+    for (int c0 = 0; c0 < nsrc; c0 += bd) {
+      const int k = c0 + tid;
+      const int m = (k < nsrc && mf[k]) ? bst[k] : -1;
+      const unsigned same = __match_any_sync(0xffffffffu, m);
+      const int rank = __popc(same & lt), cnt = __popc(same);
+      for (int w = 0; w < (bd >> 5); ++w) {
+        if ((tid >> 5) == w) {
+          const int base = m >= 0 ? cur[m] : 0;
+          __syncwarp();
+          if (m >= 0) {
+            mem[base + rank] = k;
+            if (rank == 0) cur[m] = base + cnt;
+          }
+        }
+        __syncthreads();
+      }
+    }
+  } else {
+    for (int k = tid; k < nsrc; k += bd)
+      if (mf[k]) aux[atomicAdd(&cur[bst[k]], 1)] = k;
+  }
   {
     // kept sources in ascending ordinal after the r merged ones
     uint32_t nm = 0;
@@ -240,12 +275,14 @@ plan_kernel(Dims dims, const BlockDesc* __restrict__ blocks, Buffers buf, Debug 
     }
   }
   __syncthreads();
-  for (int p = tid; p < r; p += bd) {
-    const int v = aux[p];
-    const int m = bst[v], s0 = gsm[m], c = cm[m];
-    int rank = 0;
-    for (int j = 0; j < c; ++j) rank += aux[s0 + j] < v;
-    mem[s0 + rank] = v;
+  if (!big_groups) {
+    for (int p = tid; p < r; p += bd) {
+      const int v = aux[p];
+      const int m = bst[v], s0 = gsm[m], c = cm[m];
+      int rank = 0;
+      for (int j = 0; j < c; ++j) rank += aux[s0 + j] < v;
+      mem[s0 + rank] = v;
+    }
   }
   __syncthreads();
 
