@@ -8,6 +8,7 @@ from .binding import (  # noqa: F401
     HTTM_DENSE,
     HTTM_HEAD_UNIFORM,
     HTTM_HEADWISE_TEMPORAL,
+    HTTM_PARTITION,
     HttmError,
     TorchExchange,
     LayerConfig,
@@ -20,7 +21,9 @@ from .binding import (  # noqa: F401
     httm_forward_with_plan,
     httm_get_device_status,
     httm_plan,
+    httm_plan_partition,
     httm_reorder,
+    httm_set_fused_unmerge,
     httm_set_wait_budget,
     load_library,
     workspace_view,
