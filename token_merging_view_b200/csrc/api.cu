@@ -158,6 +158,8 @@ Workspace layout(const Dims& d, bool fp32) {
   w.k_members = take(hN * 4);
   w.k_gstart = take((size_t)d.h * d.k_slots * 4);
   w.k_gcount = take((size_t)d.h * d.k_slots * 4);
+  w.q_big = take(big_list_cap(d.h, d.N) * 4);
+  w.k_big = take(big_list_cap(d.h, d.N) * 4);
   w.q_tilde = take((size_t)d.q_rows_alloc * d.d * es);
   w.k_tilde = take((size_t)d.h * d.k_slots * d.d * es);
   w.v_tilde = take((size_t)d.h * d.k_slots * d.d * es);
@@ -193,6 +195,8 @@ Buffers resolve(const Workspace& w, void* base) {
   b.k_members = reinterpret_cast<int32_t*>(p + w.k_members);
   b.k_gstart = reinterpret_cast<int32_t*>(p + w.k_gstart);
   b.k_gcount = reinterpret_cast<int32_t*>(p + w.k_gcount);
+  b.q_big = reinterpret_cast<int32_t*>(p + w.q_big);
+  b.k_big = reinterpret_cast<int32_t*>(p + w.k_big);
   b.q_tilde = p + w.q_tilde;
   b.k_tilde = p + w.k_tilde;
   b.v_tilde = p + w.v_tilde;
@@ -317,7 +321,7 @@ httm_status filter_stage(const httm_plan_s* plan, const void* Q, bool mask_inj, 
     *launches += 2;  // scan, emit
   }
   if (cudaError_t e_ = checked(launch_restore(dims, fp32, plan->blocks_d, Q, buf, dd, s), s); e_ != cudaSuccess) return cuda_fail(e_, "launch_restore");
-  ++*launches;
+  *launches += 2;  // the restore, then its big slots
   return HTTM_OK;
 }
 
@@ -389,7 +393,7 @@ httm_status forward_impl(httm_plan_s* plan, const void* Q, const void* K, const 
     }
     HTTM_LAUNCH(launch_merge(dims, fp32, plan->blocks_d, plan_inj, reuse, Q, K, V, buf, dd, s, 1));
     HTTM_LAUNCH(launch_merge(dims, fp32, plan->blocks_d, plan_inj, reuse, Q, K, V, buf, dd, s2, 2));
-    if (!reuse) launches += 2;  // the two planning launches
+    launches += reuse ? 2 : 4;  // the big-slot kernels after both gathers, and (unless reused) both plannings
     if ((st = filter_stage(plan, Q, mask_inj, buf, dd, s, ex, &launches)) != HTTM_OK) return st;
     if (cudaEventRecord(plan->ev_join, s2) != cudaSuccess || cudaStreamWaitEvent(s, plan->ev_join, 0) != cudaSuccess)
       return HTTM_ERR_CUDA;
@@ -414,9 +418,9 @@ httm_status forward_impl(httm_plan_s* plan, const void* Q, const void* K, const 
     if (e != cudaSuccess) return cuda_fail(e, "matching");
   }
   {
-    StageTimer t(plan, s, HTTM_STAGE_MERGE, reuse ? 2 : 3);
+    StageTimer t(plan, s, HTTM_STAGE_MERGE, reuse ? 4 : 5);
     HTTM_LAUNCH(launch_merge(dims, fp32, plan->blocks_d, plan_inj, reuse, Q, K, V, buf, dd, s));
-    launches += reuse ? 1 : 2;  // planning (unless reused), then the two gathers
+    launches += reuse ? 3 : 4;  // planning (unless reused), then each gather and its big-slot kernel
   }
   {
     const int before = launches;

@@ -56,8 +56,13 @@ constexpr int kHistBins = 2048;    // radix digit of the outlier select (11 bits
 constexpr int kMaxShards = 64;     // head shards of one layer (httm_plan_shard)
 constexpr int kAttnRows = 256;     // query rows per attention work item (two 128-row tiles)
 constexpr int kMaxAttnParts = 256; // partial results of the last wave's split items (<= one per SM)
+constexpr int kBigSlot = 32;       // slots with more members are summed by a whole CTA (listed, then a kernel of their own)
 constexpr int kAttnPartStride = 68; // floats per partial row: O (64), row sum, max in use, 2 unused (16-byte rows)
 static_assert(kAttnPartStride * 4 % 16 == 0, "partial rows are read and written as float4");
+
+// Capacity of the list of big query slots: members of the slots of one head
+// are distinct tokens, so a head has at most N / (kBigSlot + 1) of them.
+constexpr size_t big_list_cap(int h, int N) { return (size_t)h * ((size_t)N / (kBigSlot + 1) + 1); }
 
 // Device-side state at the head of the workspace.
 struct DevState {
@@ -69,14 +74,15 @@ struct DevState {
   uint32_t wait_site;            // first bounded wait that ran out: barrier offset | parity << 20 | 1 << 31
   uint32_t wait_cta;             // ... its CTA index
   uint32_t wait_grid;            // ... and the grid size of its launch (tells the kernels apart)
-  uint32_t pad_;
+  uint32_t n_big;                // query slots listed in Buffers::q_big
+  uint32_t n_kbig;               // key slots listed in Buffers::k_big
   uint64_t wait_ns;              // this call's wait bound (from Dims::wait_budget_ns)
 };
 
 struct Workspace {
   size_t state, hist, chunk, n_out, out_base, items;
   size_t q_best, q_score, q_merged, k_best, k_score, k_merged;
-  size_t q_slot, q_orank, o_tok, keys, mask, q_members, q_gstart, q_gcount, k_members, k_gstart, k_gcount;
+  size_t q_slot, q_orank, o_tok, keys, mask, q_members, q_gstart, q_gcount, k_members, k_gstart, k_gcount, q_big, k_big;
   size_t q_tilde, k_tilde, v_tilde, o_tilde;
   size_t attn_part;
   size_t total;
@@ -105,6 +111,8 @@ struct Buffers {
   int32_t* k_members;      // the same for the key plan (values follow it)
   int32_t* k_gstart;
   int32_t* k_gcount;
+  int32_t* q_big;          // [big_list_cap]: the query slots of more than kBigSlot members, any order
+  int32_t* k_big;          // the same for the key slots
   void* q_tilde; void* k_tilde; void* v_tilde; void* o_tilde;
   float* attn_part;        // [kMaxAttnParts][kAttnRows][kAttnPartStride]: partial attention of split items
 };

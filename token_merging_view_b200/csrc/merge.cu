@@ -13,7 +13,9 @@
 // (~order(score), source ordinal), so ties go to the lower in-block index;
 // the groups come from a second sort of (best destination, source ordinal),
 // which lists every group's members in ascending order.  Sums accumulate in
-// fp32 in member order (destination first), so results are bit-reproducible.
+// fp32 in member order (destination first), or for a slot of more than
+// kBigSlot members in a fixed split over a CTA's row groups, so results are
+// bit-reproducible.
 #include <algorithm>
 
 #include "common.cuh"
@@ -296,6 +298,10 @@ plan_kernel(Dims dims, const BlockDesc* __restrict__ blocks, Buffers buf, Debug 
     gstart[slot_off + m] = b.tok_off + p0;
     gcount[slot_off + m] = c;
     for (int j = 0; j < c; ++j) pm[p0 + j] = m;
+    if (c > kBigSlot) {                              // a big slot: listed for the CTA-wide kernels
+      const uint32_t k = atomicAdd(is_q ? &buf.state->n_big : &buf.state->n_kbig, 1u);
+      if (k < big_list_cap(dims.h, dims.N)) (is_q ? buf.q_big : buf.k_big)[k] = hh * nslots + slot_off + m;
+    }
   }
   for (int p = tid; p < nsrc - r; p += bd) {
     gstart[slot_off + ndst + p] = b.tok_off + ndst + r + p;
@@ -327,6 +333,71 @@ plan_kernel(Dims dims, const BlockDesc* __restrict__ blocks, Buffers buf, Debug 
   }
 }
 
+// Slots with more than kBigSlot members -- a destination that drew most of
+// its block, as near-identical tokens make it -- are not left to one row
+// group, whose member loop would take c / kU dependent steps: the row-group
+// kernels list them, and a kernel launched after them gives each listed slot
+// a whole CTA.  Row group g of the CTA's RG adds the members g, g + RG,
+// g + 2 RG, ... in that order, and the partial rows are then added in
+// row-group order, element by element: a fixed order, so the result is
+// reproducible (and the same wherever a slot is summed this way).
+
+template <class T, int D>
+struct SlotCta {
+  using Ch = Chunk<T, D>;
+  static constexpr int RG = (256 / 32) * Ch::RPI;   // row groups of a 256-thread CTA
+};
+
+// sum[t * D + e] = sum over the members q < c of mem with use(q, tok) of row
+// tok of tensor t (NT tensors), by all 256 threads of the CTA.  part holds
+// NT * RG * D floats and sum NT * D (shared memory); the sums are visible to
+// every thread on return.
+template <class T, int D, int NT, class Use>
+__device__ void cta_slot_sum(const T* const (&X)[NT], const int32_t* mem, int c, Use use, float* part, float* sum) {
+  using Ch = Chunk<T, D>;
+  constexpr int CPR = Ch::CPR, EPC = Ch::EPC, RG = SlotCta<T, D>::RG, kU = 4;
+  const int lane = threadIdx.x & 31;
+  const int g = (int)(threadIdx.x >> 5) * Ch::RPI + lane / CPR, ch = lane % CPR;
+  float acc[NT][EPC];
+#pragma unroll
+  for (int t = 0; t < NT; ++t)
+#pragma unroll
+    for (int e = 0; e < EPC; ++e) acc[t][e] = 0.f;
+  for (int q0 = g; q0 < c; q0 += kU * RG) {
+    uint4 x[NT][kU];
+    bool on[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int q = q0 + u * RG;
+      on[u] = false;
+      if (q < c) {
+        const int tok = mem[q];
+        on[u] = use(q, tok);
+        if (on[u])
+#pragma unroll
+          for (int t = 0; t < NT; ++t) x[t][u] = Ch::load(X[t] + (size_t)tok * D, ch);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kU; ++u)
+      if (on[u])
+#pragma unroll
+        for (int t = 0; t < NT; ++t) Ch::add(acc[t], x[t][u]);
+  }
+#pragma unroll
+  for (int t = 0; t < NT; ++t)
+#pragma unroll
+    for (int e = 0; e < EPC; ++e) part[(t * RG + g) * D + ch * EPC + e] = acc[t][e];
+  __syncthreads();
+  for (int i = threadIdx.x; i < NT * D; i += blockDim.x) {
+    const int t = i / D, e = i - t * D;
+    float v = 0.f;
+    for (int r = 0; r < RG; ++r) v += part[(t * RG + r) * D + e];
+    sum[i] = v;
+  }
+  __syncthreads();
+}
+
 // Mean merging (key design 1), flat over every (head, slot).  Rows are read
 // as 16-byte chunks, lane l owning chunk l % CPR; each of the RPI row groups
 // of a warp (CPR lanes) takes its own slot, fetches up to kU member rows
@@ -335,7 +406,9 @@ plan_kernel(Dims dims, const BlockDesc* __restrict__ blocks, Buffers buf, Debug 
 // lookups overlap the row loads.  Queries also get each member's deviation
 // from the mean (key design 3), kept as a 32-bit key (bits(dev) + 1 for
 // members of groups of >= 2, else 0), and the first radix digit of those
-// keys is histogrammed for the global outlier select.
+// keys is histogrammed for the global outlier select.  A slot of more than
+// kBigSlot members (the planning lists them in Buffers::q_big / k_big) is
+// left to big_gather_kernel.
 template <class T, int D, bool IS_Q>
 __global__ void __launch_bounds__(256, 4)
 gather_kernel(Dims dims, const T* __restrict__ X, const T* __restrict__ V, Buffers buf, Debug dbg, int reuse) {
@@ -375,6 +448,7 @@ gather_kernel(Dims dims, const T* __restrict__ X, const T* __restrict__ V, Buffe
     if (gsl < total) {
       c = gcount[gsl];
       gs = gstart[gsl];
+      if (c > kBigSlot) c = 0;                     // big_gather_kernel's (the planning listed it)
       const size_t tb = (size_t)(gsl / nslots) * dims.N;
 #pragma unroll
       for (int u = 0; u < kU; ++u) tk[u] = u < c ? members[tb + gs + u] : 0;
@@ -434,7 +508,7 @@ gather_kernel(Dims dims, const T* __restrict__ X, const T* __restrict__ V, Buffe
           }
         }
       }
-      const bool live = gsl < total;
+      const bool live = gsl < total && c_cur > 0;
       if (live) {
         const float inv = 1.f / (float)c_cur;
 #pragma unroll
@@ -517,6 +591,104 @@ gather_kernel(Dims dims, const T* __restrict__ X, const T* __restrict__ V, Buffe
   }
 }
 
+// The slots the gather listed as big (more than kBigSlot members), one at a
+// time per CTA: the mean by cta_slot_sum and, for queries, every member's
+// deviation key and its first radix digit, as in gather_kernel.
+template <class T, int D, bool IS_Q>
+__global__ void __launch_bounds__(256)
+big_gather_kernel(Dims dims, const T* __restrict__ X, const T* __restrict__ V, Buffers buf, Debug dbg) {
+  using Ch = Chunk<T, D>;
+  constexpr int CPR = Ch::CPR, RPI = Ch::RPI, EPC = Ch::EPC, NT = IS_Q ? 1 : 2, RG = SlotCta<T, D>::RG, kU = 4;
+  const uint32_t listed = *(volatile const uint32_t*)(IS_Q ? &buf.state->n_big : &buf.state->n_kbig);
+  const int nbig = (int)min(listed, (uint32_t)big_list_cap(dims.h, dims.N));
+  if ((int)blockIdx.x >= nbig) return;
+  if (cta_plan_failed(buf.state)) return;
+  __shared__ uint32_t hist[IS_Q ? kHistBins : 1];
+  __shared__ uint32_t s_elig;
+  __shared__ float s_part[NT * RG * D], s_sum[NT * D];
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int ch = lane % CPR, g = (tid >> 5) * RPI + lane / CPR;
+  if (IS_Q) {
+    for (int i = tid; i < kHistBins; i += blockDim.x) hist[i] = 0;
+    if (tid == 0) s_elig = 0;
+    __syncthreads();
+  }
+  const int nslots = IS_Q ? dims.q_slots : dims.k_slots;
+  const int total = dims.h * nslots;
+  const int32_t* list = IS_Q ? buf.q_big : buf.k_big;
+  const int32_t* members = IS_Q ? buf.q_members : buf.k_members;
+  const int32_t* gstart = IS_Q ? buf.q_gstart : buf.k_gstart;
+  const int32_t* gcount = IS_Q ? buf.q_gcount : buf.k_gcount;
+  T* Xt = reinterpret_cast<T*>(IS_Q ? buf.q_tilde : buf.k_tilde);
+  T* Vt = reinterpret_cast<T*>(buf.v_tilde);
+  float* dmean = IS_Q ? dbg.q_means : dbg.k_means;
+  uint32_t elig = 0;
+  for (int i = blockIdx.x; i < nbig; i += gridDim.x) {
+    const int gsl = list[i];
+    if (gsl < 0 || gsl >= total) {
+      if (tid == 0) set_status(buf.state, HTTM_DEV_BOUNDS);
+      continue;
+    }
+    const size_t tokbase = (size_t)(gsl / nslots) * dims.N;
+    const int c = gcount[gsl];
+    const int32_t* mem = members + tokbase + gstart[gsl];
+    if constexpr (IS_Q) {
+      const T* const src[1] = {X + tokbase * D};
+      cta_slot_sum<T, D, 1>(src, mem, c, [](int, int) { return true; }, s_part, s_sum);
+    } else {
+      const T* const src[2] = {X + tokbase * D, V + tokbase * D};
+      cta_slot_sum<T, D, 2>(src, mem, c, [](int, int) { return true; }, s_part, s_sum);
+    }
+    const float inv = 1.f / (float)c;
+    float mean[EPC], meanv[EPC];
+#pragma unroll
+    for (int e = 0; e < EPC; ++e) {
+      mean[e] = s_sum[ch * EPC + e] * inv;
+      meanv[e] = s_sum[(NT - 1) * D + ch * EPC + e] * inv;
+    }
+    if (g == 0) {
+      Ch::store(Xt + (size_t)gsl * D, ch, mean);
+      if (dmean) Ch::store_f32(dmean + (size_t)gsl * D, ch, mean);
+      if (!IS_Q) {
+        Ch::store(Vt + (size_t)gsl * D, ch, meanv);
+        if (dbg.v_means) Ch::store_f32(dbg.v_means + (size_t)gsl * D, ch, meanv);
+      }
+    }
+    if (IS_Q) {
+      // every member's deviation from the mean (c > kBigSlot >= 2: all eligible)
+      const T* Xh = X + tokbase * D;
+      for (int q0 = 0; q0 < c; q0 += kU * RG) {
+        uint4 x[kU];
+        int tok[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          const int q = q0 + u * RG + g;
+          tok[u] = q < c ? mem[q] : -1;
+          if (tok[u] >= 0) x[u] = Ch::load(Xh + (size_t)tok[u] * D, ch);
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          const float ss = Ch::within_row(tok[u] >= 0 ? Ch::sq_dist(x[u], mean) : 0.f);
+          if (tok[u] >= 0 && ch == 0) {
+            const uint32_t key = __float_as_uint(sqrtf(ss)) + 1u;
+            buf.keys[tokbase + tok[u]] = key;
+            atomicAdd(&hist[key >> 21], 1u);
+            ++elig;
+          }
+        }
+      }
+    }
+    __syncthreads();                                   // s_sum is the next slot's
+  }
+  if (IS_Q) {
+    if (elig) atomicAdd(&s_elig, elig);
+    __syncthreads();
+    for (int i = tid; i < kHistBins; i += blockDim.x)
+      if (hist[i]) atomicAdd(&buf.hist[i], hist[i]);
+    if (tid == 0 && s_elig) atomicAdd(&buf.state->n_eligible, s_elig);
+  }
+}
+
 // Restore (key design 3), flat over every (head, query slot): a slot holding
 // outliers becomes the mean of its remaining members (in member order); a
 // slot whose members are all outliers is drained (zeros; no token reads it).
@@ -543,6 +715,7 @@ restore_kernel(Dims dims, const T* __restrict__ Q, Buffers buf, Debug dbg) {
       if (ch == 0) set_status(buf.state, HTTM_DEV_BOUNDS);
       c = 0;
     }
+    if (c > kBigSlot) c = 0;                           // restore_big_kernel takes it
     // outliers among the members (the lanes of the row group share them out)
     int nout = 0;
     if (c >= 2) {
@@ -596,6 +769,7 @@ restore_kernel(Dims dims, const T* __restrict__ Q, Buffers buf, Debug dbg) {
 // recomputes the slot's mean from the remaining members -- the same members
 // in the same order, added the same way as the flat kernel above, so both
 // give the same bits; a slot whose members are all outliers is drained.
+// Big slots are restore_big_kernel's, after either kernel.
 template <class T, int D>
 __global__ void __launch_bounds__(256)
 restore_out_kernel(Dims dims, const T* __restrict__ Q, Buffers buf) {
@@ -637,6 +811,7 @@ restore_out_kernel(Dims dims, const T* __restrict__ Q, Buffers buf) {
         if (ch == 0) set_status(buf.state, HTTM_DEV_BOUNDS);
         c = 0;
       }
+      if (c > kBigSlot) c = 0;                         // restore_big_kernel takes it
     }
     // outliers among the members, and the first of them in member order
     int nout = 0, first = 0x7fffffff;
@@ -679,6 +854,71 @@ restore_out_kernel(Dims dims, const T* __restrict__ Q, Buffers buf) {
 #pragma unroll
     for (int e = 0; e < EPC; ++e) acc[e] = remain ? acc[e] / (float)remain : 0.f;
     Ch::store(Qt + (size_t)gsl * D, ch, acc);
+  }
+}
+
+// The big query slots (more than kBigSlot members; the query gather listed
+// them), one at a time per CTA: the outliers among the members, then the sum
+// of the others as cta_slot_sum adds them, divided by their count -- the
+// slot's new row when it holds outliers.  dbg_rows (the fp32 export, or null)
+// gets that mean for every big slot (NaN where every member is an outlier).
+template <class T, int D>
+__global__ void __launch_bounds__(256)
+restore_big_kernel(Dims dims, const T* __restrict__ Q, Buffers buf, float* dbg_rows) {
+  using Ch = Chunk<T, D>;
+  constexpr int CPR = Ch::CPR, EPC = Ch::EPC, RG = SlotCta<T, D>::RG;
+  const uint32_t listed = *(volatile const uint32_t*)&buf.state->n_big;
+  const int nbig = (int)min(listed, (uint32_t)big_list_cap(dims.h, dims.N));
+  if ((int)blockIdx.x >= nbig) return;
+  if (cta_plan_failed(buf.state)) return;
+  if (buf.state->sel[3] == 0 && dbg_rows == nullptr) return;     // no outlier anywhere
+  __shared__ float s_part[RG * D], s_sum[D];
+  const int lane = threadIdx.x & 31, ch = lane % CPR;
+  const int g = (int)(threadIdx.x >> 5) * Ch::RPI + lane / CPR;
+  T* Qt = reinterpret_cast<T*>(buf.q_tilde);
+  const int total = dims.h * dims.q_slots;
+  for (int i = blockIdx.x; i < nbig; i += gridDim.x) {
+    const int gsl = buf.q_big[i];
+    int c = 0, gs = 0, hh = 0;
+    if (gsl >= 0 && gsl < total) {
+      hh = gsl / dims.q_slots;
+      c = buf.q_gcount[gsl];
+      gs = buf.q_gstart[gsl];
+    }
+    if (gsl < 0 || gsl >= total || c < 0 || gs < 0 || gs + c > dims.N) {
+      if (threadIdx.x == 0) set_status(buf.state, HTTM_DEV_BOUNDS);
+      c = 0;
+    }
+    const size_t tokbase = (size_t)hh * dims.N;
+    const int32_t* mem = buf.q_members + tokbase + gs;
+    int nout = 0;
+    for (int q0 = 0; q0 < c; q0 += blockDim.x) {
+      const int q = q0 + threadIdx.x;
+      bool o = false;
+      if (q < c) {
+        const int tok = mem[q];
+        o = tok >= 0 && tok < dims.N && buf.mask[tokbase + tok] != 0;
+      }
+      nout += __syncthreads_count(o);
+    }
+    if (c == 0 || (nout == 0 && dbg_rows == nullptr)) continue;
+    const T* const src[1] = {Q + tokbase * D};
+    cta_slot_sum<T, D, 1>(
+        src, mem, c,
+        [&](int, int tok) { return tok >= 0 && tok < dims.N && buf.mask[tokbase + tok] == 0; }, s_part, s_sum);
+    const int remain = c - nout;
+    if (g == 0) {
+      float acc[EPC];
+#pragma unroll
+      for (int e = 0; e < EPC; ++e) acc[e] = remain ? s_sum[ch * EPC + e] / (float)remain : 0.f;
+      if (nout > 0) Ch::store(Qt + (size_t)gsl * D, ch, acc);
+      if (dbg_rows) {
+#pragma unroll
+        for (int e = 0; e < EPC; ++e) acc[e] = remain ? acc[e] : __int_as_float(0x7fc00000);
+        Ch::store_f32(dbg_rows + (size_t)gsl * D, ch, acc);
+      }
+    }
+    __syncthreads();                                   // s_sum is the next slot's
   }
 }
 
@@ -779,6 +1019,10 @@ __global__ void zero_state_kernel(Buffers buf, int keep_stamp, unsigned long lon
     buf.state->wait_site = 0u;
     buf.state->wait_cta = 0u;
     buf.state->wait_grid = 0u;
+    if (!keep_stamp) {                             // the big-slot lists go with the member lists
+      buf.state->n_big = 0u;
+      buf.state->n_kbig = 0u;
+    }
     buf.state->wait_ns = wait_ns;
   }
   if (threadIdx.x < 8) buf.state->sel[threadIdx.x] = 0u;
@@ -807,12 +1051,19 @@ cudaError_t launch_merge_t(const Dims& dims, const BlockDesc* blocks, bool injec
   }
   constexpr int RPI = Chunk<T, D>::RPI;
   // resident warps handle several slots each, so that prefetching pays
-  if (do_q)
+  // the big slots' kernels: as many CTAs as the lists could need, at most
+  // two per SM; CTAs past the listed count return at once
+  const int big_grid = (int)std::min<size_t>(2 * 148, big_list_cap(dims.h, dims.N));
+  if (do_q) {
     gather_kernel<T, D, true><<<gather_grid((long long)dims.h * dims.q_slots / (4 * RPI) + 1, 4), 256, 0, s>>>(
         dims, (const T*)Q, nullptr, buf, dbg, reuse ? 1 : 0);
-  if (do_k)
+    big_gather_kernel<T, D, true><<<big_grid, 256, 0, s>>>(dims, (const T*)Q, nullptr, buf, dbg);
+  }
+  if (do_k) {
     gather_kernel<T, D, false><<<gather_grid((long long)dims.h * dims.k_slots / (4 * RPI) + 1, 4), 256, 0, s>>>(
         dims, (const T*)K, (const T*)V, buf, dbg, reuse ? 1 : 0);
+    big_gather_kernel<T, D, false><<<big_grid, 256, 0, s>>>(dims, (const T*)K, (const T*)V, buf, dbg);
+  }
   return cudaGetLastError();
 }
 
@@ -841,11 +1092,13 @@ cudaError_t launch_restore(const Dims& dims, bool fp32, const BlockDesc*, const 
   // otherwise only the slots holding outliers change
   const bool flat = dbg.q_restored != nullptr;
   const long long units = flat ? (long long)dims.h * dims.q_slots : dims.q_rows_alloc - dims.out_base;
+  const int big_grid = (int)std::min<size_t>(2 * 148, big_list_cap(dims.h, dims.N));
 #define HTTM_RESTORE(T, DD)                                                                                  \
   do {                                                                                                       \
     const int grid = gather_grid(units / Chunk<T, DD>::RPI + 1);                                             \
     if (flat) restore_kernel<T, DD><<<grid, 256, 0, s>>>(dims, (const T*)Q, buf, dbg);                       \
     else restore_out_kernel<T, DD><<<grid, 256, 0, s>>>(dims, (const T*)Q, buf);                             \
+    restore_big_kernel<T, DD><<<big_grid, 256, 0, s>>>(dims, (const T*)Q, buf, flat ? dbg.q_restored : nullptr); \
   } while (0)
   if (fp32) {
     if (dims.d == 16) HTTM_RESTORE(float, 16);
