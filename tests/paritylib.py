@@ -227,3 +227,36 @@ def run(plan: B.Plan, Q, K, V, injected=None, debug=True, fields=None):
         out = B.httm_forward(plan, Q, K, V, workspace=ws)
     status = B.httm_get_device_status(plan, ws)
     return out, (cpu(dbg) if debug else None), ws, status
+
+
+def plant_big_groups(w: Workload, Q, K, V):
+    """Near-copies of every block's first destination: about 60 % of each
+    block's sources (the same tokens in Q and K, every head) become that
+    destination's row plus Gaussian noise of a per-token size in [0.02, 1.2]
+    (rows have unit-variance entries), so that the destination's group draws
+    far more than 32 members and its noisiest members have the largest
+    deviations of the layer (the outliers)."""
+    cfg = oracle_cfg(w)
+    assert cfg.q_stride == cfg.kv_stride
+    g = torch.Generator().manual_seed(w.seed + 101)
+    picks = []
+    for toks in O.block_list(cfg):
+        src = toks[np.arange(toks.shape[0]) % cfg.q_stride != 0]
+        keep = torch.rand(src.shape[0], generator=g).numpy() < 0.6
+        picks.append((int(toks[0]), torch.from_numpy(src[keep])))
+    for X in (Q, K):
+        Xc = X.float().cpu()
+        for d0, pick in picks:
+            eps = 0.02 + 1.18 * torch.rand(pick.shape[0], generator=g)
+            noise = torch.randn(w.h, pick.shape[0], w.d, generator=g)
+            Xc[:, pick] = Xc[:, d0][:, None, :] + eps[None, :, None] * noise
+        X.copy_(Xc.to(X.dtype))
+
+
+def group_sizes(plan: O.TensorPlan) -> np.ndarray:
+    """Members per group (the destination itself included), per head."""
+    out = []
+    for hh in range(plan.best.shape[0]):
+        dst = plan.best[hh][plan.merged[hh]]
+        out.append(np.bincount(dst, minlength=plan.best.shape[1]) + plan.is_dst)
+    return np.stack(out)

@@ -171,39 +171,6 @@ def test_dense_mode_and_unmerged_layer():
     assert np.abs(g0 - want).max() <= PL.OUT_MAX_ABS
 
 
-def _plant_big_groups(w: Workload, Q, K, V):
-    """Near-copies of every block's first destination: about 60 % of each
-    block's sources (the same tokens in Q and K, every head) become that
-    destination's row plus Gaussian noise of a per-token size in [0.02, 1.2]
-    (rows have unit-variance entries), so that the destination's group draws
-    far more than 32 members and its noisiest members have the largest
-    deviations of the layer (the outliers)."""
-    cfg = PL.oracle_cfg(w)
-    assert cfg.q_stride == cfg.kv_stride
-    g = torch.Generator().manual_seed(w.seed + 101)
-    picks = []
-    for toks in O.block_list(cfg):
-        src = toks[np.arange(toks.shape[0]) % cfg.q_stride != 0]
-        keep = torch.rand(src.shape[0], generator=g).numpy() < 0.6
-        picks.append((int(toks[0]), torch.from_numpy(src[keep])))
-    for X in (Q, K):
-        Xc = X.float().cpu()
-        for d0, pick in picks:
-            eps = 0.02 + 1.18 * torch.rand(pick.shape[0], generator=g)
-            noise = torch.randn(w.h, pick.shape[0], w.d, generator=g)
-            Xc[:, pick] = Xc[:, d0][:, None, :] + eps[None, :, None] * noise
-        X.copy_(Xc.to(X.dtype))
-
-
-def _group_sizes(plan: O.TensorPlan) -> np.ndarray:
-    """Members per group (the destination itself included), per head."""
-    out = []
-    for hh in range(plan.best.shape[0]):
-        dst = plan.best[hh][plan.merged[hh]]
-        out.append(np.bincount(dst, minlength=plan.best.shape[1]) + plan.is_dst)
-    return np.stack(out)
-
-
 @pytest.mark.parametrize("kw", [dict(), dict(out_pct=100)], ids=["d10", "d100"])
 def test_big_groups(kw):
     """Groups of more than 32 members (a destination that draws most of its
@@ -211,11 +178,11 @@ def test_big_groups(kw):
     against the oracle, as in the other layers, with big groups in both plans
     and outliers among their members."""
     def check(res):
-        qs, ks = _group_sizes(res.q_plan), _group_sizes(res.k_plan)
+        qs, ks = PL.group_sizes(res.q_plan), PL.group_sizes(res.k_plan)
         assert (qs > 32).sum() >= 20 and (ks > 32).sum() >= 20, ((qs > 32).sum(), (ks > 32).sum())
         big = np.take_along_axis(qs, np.maximum(res.q_plan.best, 0), axis=1) > 32
         assert (res.mask & big).sum() > 0
-    _full_check(MID.with_(**kw) if kw else MID, transform=_plant_big_groups, inspect=check)
+    _full_check(MID.with_(**kw) if kw else MID, transform=PL.plant_big_groups, inspect=check)
 
 
 def test_identical_and_zero_tokens():

@@ -97,6 +97,28 @@ def test_reuse_equals_forward_with_the_same_plan():
     assert torch.equal(out_r, out_p)
 
 
+def test_reuse_keeps_the_big_group_lists():
+    """Groups of more than 32 members are summed by kernels of their own
+    from lists the planning writes; a reusing call plans nothing and takes
+    them from the workspace with the member lists.  Its output equals that
+    of the same plan passed in (which plans, and lists, afresh)."""
+    w = MID
+    plan, cfg, X1 = _setup(w)
+    PL.plant_big_groups(w, *X1)
+    dbg = B.debug_buffers(plan)
+    ws = plan.new_workspace()
+    B.httm_forward_debug(plan, *X1, dbg, workspace=ws)
+    assert B.httm_get_device_status(plan, ws) == 0
+    counts = np.stack([np.bincount(row, minlength=w.N) for row in dbg["q_slot"].cpu().numpy()])
+    assert (counts > 32).sum() >= 20
+    X2 = _next_layer(w, X1, 9)
+    out_r = B.httm_forward_reuse(plan, *X2, workspace=ws)
+    assert B.httm_get_device_status(plan, ws) == 0
+    inj = {k: dbg[k] for k in ("q_best", "q_merged", "k_best", "k_merged")}
+    out_p = B.httm_forward_with_plan(plan, *X2, inj, workspace=plan.new_workspace())
+    assert torch.equal(out_r, out_p)
+
+
 def test_reuse_without_member_lists_sets_status():
     w = MID.with_(T=3, h=2)
     plan, cfg, X1 = _setup(w)

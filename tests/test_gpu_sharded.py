@@ -136,6 +136,18 @@ def test_sharded_layer_equals_unsharded(w, shards):
     check_against_unsharded(w, shards, Q, K, V)
 
 
+@pytest.mark.parametrize("shards", [2, 4])
+def test_sharded_big_groups_equal_unsharded(shards):
+    """Groups of more than 32 members (each shard lists its own heads' and
+    sums them with the CTA-wide kernels): the same masks, slots and
+    exports as the unsharded layer."""
+    Q, K, V = PL.inputs(MID)
+    PL.plant_big_groups(MID, Q, K, V)
+    dbg, _ = check_against_unsharded(MID, shards, Q, K, V)
+    counts = np.stack([np.bincount(row, minlength=MID.N) for row in dbg["q_slot"]])
+    assert (counts > 32).sum() >= 20
+
+
 def test_sharded_ties_are_taken_in_flat_index_order():
     """Q all zero: every eligible query deviates by 0, so the whole budget
     (40 % of h N here) is one tie, taken in flat-index order: every eligible
