@@ -548,7 +548,9 @@ def run_ours(args):
         line = {
             "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            # one GPU: the first point of the head-sharded series (one layer split
+            # over the ranks, total work fixed); replicas on several GPUs: weak
+            "higher_is_better": True, "scaling": "strong" if world == 1 else "weak", "vs_baseline": None,
             "dtype": "f32" if w.fp32 else "bf16",
             "data": "synthetic (seeded blurred-field Q/K/V, VGGT global-attention shapes)",
             "config": workload_config(w, world),
