@@ -13,8 +13,9 @@
 //               layout (all destinations of the block once, then source tiles
 //               double-buffered), compute norms, and run the epilogue: warp w
 //               reads TMEM lanes 32*(w%4).. (one source row per thread) and the
-//               32-column groups g = w/4, w/4 + 4, ... of each chunk (both of
-//               its loads in flight at once); running (max, first index).
+//               32-column groups g = w/4, w/4 + 4, ... of each chunk, one
+//               group's load at a time (a second group in registers spills);
+//               running (max, first index).
 //               Four warps per TMEM lane quarter keep the argmax, the bound of
 //               this kernel (a multiply, compare and two selects per score),
 //               issuing while others wait on TMEM or the MMA;
