@@ -17,7 +17,8 @@
 //               group's load at a time (a second group in registers spills);
 //               running (max, first index).
 //               Four warps per TMEM lane quarter keep the argmax, the bound of
-//               this kernel (a multiply, compare and two selects per score),
+//               this kernel (half a packed multiply, a compare and two
+//               selects per score),
 //               issuing while others wait on TMEM or the MMA;
 //   warp 16     allocates TMEM and one thread issues tcgen05.mma: for each
 //               source tile, destination chunks of <= 256 columns into two
@@ -238,8 +239,13 @@ match_tc_kernel(Dims dims, const BlockDesc* __restrict__ blocks, const int4* __r
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
               const float4 iv = invp[q];
-              const float v0 = __uint_as_float(r[4 * q]) * iv.x, v1 = __uint_as_float(r[4 * q + 1]) * iv.y;
-              const float v2 = __uint_as_float(r[4 * q + 2]) * iv.z, v3 = __uint_as_float(r[4 * q + 3]) * iv.w;
+              // the scaling on packed pairs: one instruction for two scores, the same products
+              float v0, v1, v2, v3;
+              f2_unpack(f2_mul(f2_pack(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1])), f2_pack(iv.x, iv.y)),
+                        v0, v1);
+              f2_unpack(f2_mul(f2_pack(__uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3])),
+                               f2_pack(iv.z, iv.w)),
+                        v2, v3);
               if (v0 > bv[0]) { bv[0] = v0; bx[0] = cb + 4 * q; }
               if (v1 > bv[1]) { bv[1] = v1; bx[1] = cb + 4 * q + 1; }
               if (v2 > bv[2]) { bv[2] = v2; bx[2] = cb + 4 * q + 2; }
