@@ -200,6 +200,57 @@ def test_identical_and_zero_tokens():
     assert np.all(dbg["dev"] == 0.0)
 
 
+@pytest.mark.slow
+def test_identical_tokens_30f_layer():
+    """The 30-frame layer with every query zero and every key of a head
+    identical (V as drawn): every cosine ties, so each block's sources all
+    take its first destination and the top-r merge takes its first r sources
+    -- one group of about 2,000 members per block, head and tensor, the case
+    the CTA-wide big-slot kernels are for.  Every query deviation is 0, so
+    the outlier budget is one tie taken in flat-index order.  The query plan,
+    the mask, the slots and the outlier counts equal the oracle's exactly
+    (zero rows make its cosines and deviations exactly 0 too); the key plan
+    equals the tie rules written out; every output row is the mean of the
+    shortened values (every score ties)."""
+    w = WORKLOADS["vggt_30f"]
+    _, plan, cfg, (Q, K, V), _ = _case(w)
+    Q = torch.zeros_like(Q)
+    K = K[:, :1].expand_as(K).contiguous()
+    q, k, v = (PL.to64(t) for t in (Q, K, V))
+    res = O.forward_plan(cfg, q, k, v)
+    out, dbg, ws, status = PL.run(plan, Q, K, V)
+    assert status == 0
+    # the key plan by the tie rules: every source to its block's first
+    # destination; the first r sources (in-block order) merged
+    blocks = O.block_list(cfg)
+    best = np.full(w.N, -1, dtype=np.int64)
+    merged = np.zeros(w.N, dtype=bool)
+    members = []                                   # the key slots' members, every head alike
+    for toks in blocks:
+        d_i, s_i = O.split_dst_src(toks.shape[0], cfg.kv_stride)
+        r = O.merge_count(toks.shape[0], cfg.kv_pct)
+        best[toks[s_i]] = toks[0]
+        merged[toks[s_i[:r]]] = True
+        members.append(np.concatenate([toks[:1], toks[s_i[:r]]]))
+        members += [toks[[i]] for i in d_i[1:]] + [toks[[i]] for i in s_i[r:]]
+    assert max(m.shape[0] for m in members) > 1000
+    assert np.array_equal(dbg["k_best"], np.broadcast_to(best, dbg["k_best"].shape))
+    assert np.array_equal(dbg["k_merged"].astype(bool), np.broadcast_to(merged, dbg["k_merged"].shape))
+    assert np.array_equal(dbg["q_best"], res.q_plan.best)
+    assert np.array_equal(dbg["q_merged"].astype(bool), res.q_plan.merged)
+    assert (PL.group_sizes(res.q_plan) > 1000).sum() >= w.h * 10
+    assert np.all(dbg["dev"] == 0.0)
+    assert np.array_equal(dbg["outlier"].astype(bool), res.mask)
+    assert np.array_equal(dbg["q_slot"], res.restore.slot_final)
+    assert np.array_equal(B.workspace_view(plan, ws, "n_out").cpu().numpy(), res.restore.n_out)
+    # Q~ is zero, so every score is 0 and every output row is the mean of V~
+    vt = np.stack([np.stack([v[hh, m].mean(axis=0) for m in members]) for hh in range(w.h)])
+    want = vt.mean(axis=1)                         # [h, d]
+    got = out.float().cpu().numpy()
+    err = np.abs(got - want[:, None, :]).max()
+    assert err <= PL.OUT_MAX_ABS, err
+
+
 def test_deterministic():
     _, plan, _, (Q, K, V), _ = _case(MID)
     a, da, _, _ = PL.run(plan, Q, K, V)
